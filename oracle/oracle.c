@@ -1,0 +1,340 @@
+/*
+ * oracle.c -- plain fp64 CPU reference for exact scaled-dot-product attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call this code;
+ * only the tests, the package's smoke check and the benchmark's CPU-baseline
+ * leg do.  It shares no code, header or constant with the CUDA library.
+ *
+ * What it computes is the plain definition that every page on FlashAttention
+ * says the method reproduces exactly:
+ *   - "FlashAttention: making attention fast by respecting the memory
+ *     hierarchy", opening paragraph and the tiling paragraph: an exact
+ *     algorithm, the same math reorganised;
+ *   - "FlashAttention: Fast and Memory-Efficient Exact Attention with
+ *     IO-Awareness", section "What FlashAttention targets": same outputs as
+ *     the naive formulation;
+ *   - "Flash Attention", sections "Definition" and "Common Confusions": exact,
+ *     not approximate attention.
+ * So the oracle is naive attention written out, in fp64, materialising every
+ * score row:
+ *     S_ij = scale * q_i . k_j          for allowed (i, j), else -inf
+ *     P_ij = exp(S_ij - m_i) / l_i      m_i = max_j S_ij, l_i = sum_j exp(S_ij - m_i)
+ *     O_i  = sum_j P_ij v_j,            LSE_i = m_i + ln l_i
+ * The per-row LSE is the "softmax normalization statistics" that the summary
+ * page's "Backward / recomputation" section says the forward stores.
+ *
+ * The backward is the calculus of that definition (the pages only say that
+ * the backward recomputes from the stored statistics):
+ *     dP_ij = dO_i . v_j,  D_i = sum_j P_ij dP_ij,  dS_ij = P_ij (dP_ij - D_i)
+ *     dV_j = sum_i P_ij dO_i,  dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i
+ *
+ * Masks: none; causal (key j visible to query i iff j <= i); block (a
+ * [nb x nb] uint8 grid of block x block tiles, 1 = keep).  A row with no
+ * allowed key has O_i = 0, LSE_i = -inf and contributes no gradient.
+ *
+ * Inputs and outputs are fp64 host arrays laid out [BH, N, d] (heads
+ * flattened), LSE and D are [BH, N].  Work is split over rows or key columns
+ * with OpenMP; every output element is written by exactly one thread, so the
+ * result does not depend on the thread count.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { OR_MASK_NONE = 0, OR_MASK_CAUSAL = 1, OR_MASK_BLOCK = 2 };
+enum { OR_OK = 0, OR_ERR_ARG = 1, OR_ERR_NOMEM = 2 };
+
+typedef struct {
+    int N, d, kind, block, nb;
+    const uint8_t *bm;
+    double scale;
+} spec_t;
+
+static int allowed(const spec_t *s, int i, int j)
+{
+    switch (s->kind) {
+    case OR_MASK_NONE: return 1;
+    case OR_MASK_CAUSAL: return j <= i;
+    default: return s->bm[(size_t)(i / s->block) * s->nb + (j / s->block)] != 0;
+    }
+}
+
+static double dot(const double *a, const double *b, int n)
+{
+    double acc = 0.0;
+#pragma omp simd reduction(+ : acc)
+    for (int k = 0; k < n; ++k) acc += a[k] * b[k];
+    return acc;
+}
+
+static int check(const spec_t *s, int BH)
+{
+    if (BH <= 0 || s->N <= 0 || s->d <= 0) return OR_ERR_ARG;
+    if (s->kind < 0 || s->kind > 2) return OR_ERR_ARG;
+    if (s->kind == OR_MASK_BLOCK && (s->bm == NULL || s->block <= 0)) return OR_ERR_ARG;
+    return OR_OK;
+}
+
+static spec_t make_spec(int N, int d, int kind, const uint8_t *bm, int block, double scale)
+{
+    spec_t s;
+    s.N = N; s.d = d; s.kind = kind; s.bm = bm; s.scale = scale;
+    s.block = block > 0 ? block : 1;
+    s.nb = (N + s.block - 1) / s.block;
+    return s;
+}
+
+/* Score row i of one head into S[0..N), masked entries -inf; returns m_i. */
+static double score_row(const spec_t *s, const double *Qh, const double *Kh, int i, double *S)
+{
+    const double *q = Qh + (size_t)i * s->d;
+    double m = -INFINITY;
+    for (int j = 0; j < s->N; ++j) {
+        if (allowed(s, i, j)) {
+            S[j] = s->scale * dot(q, Kh + (size_t)j * s->d, s->d);
+            if (S[j] > m) m = S[j];
+        } else {
+            S[j] = -INFINITY;
+        }
+    }
+    return m;
+}
+
+/* Turn a score row into probabilities in place; returns LSE_i (-inf if empty). */
+static double softmax_row(const spec_t *s, double *S, double m)
+{
+    if (m == -INFINITY) {                       /* no allowed key */
+        for (int j = 0; j < s->N; ++j) S[j] = 0.0;
+        return -INFINITY;
+    }
+    double l = 0.0;
+    for (int j = 0; j < s->N; ++j) {
+        S[j] = (S[j] == -INFINITY) ? 0.0 : exp(S[j] - m);
+        l += S[j];
+    }
+    for (int j = 0; j < s->N; ++j) S[j] /= l;
+    return m + log(l);
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Forward: O [BH,N,d], LSE [BH,N]. */
+int oracle_fwd(const double *Q, const double *K, const double *V, int BH, int N, int d,
+               int kind, const uint8_t *block_mask, int block, double scale,
+               double *O, double *LSE)
+{
+    spec_t s = make_spec(N, d, kind, block_mask, block, scale);
+    if (check(&s, BH) != OR_OK || !Q || !K || !V || !O || !LSE) return OR_ERR_ARG;
+    int err = OR_OK;
+#pragma omp parallel
+    {
+        double *P = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!P) {
+#pragma omp atomic write
+            err = OR_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 8) collapse(2)
+        for (int h = 0; h < BH; ++h)
+            for (int i = 0; i < N; ++i) {
+                if (!P) continue;
+                const size_t hoff = (size_t)h * N * d;
+                double m = score_row(&s, Q + hoff, K + hoff, i, P);
+                LSE[(size_t)h * N + i] = softmax_row(&s, P, m);
+                double *o = O + hoff + (size_t)i * d;
+                for (int k = 0; k < d; ++k) o[k] = 0.0;
+                for (int j = 0; j < N; ++j) {
+                    if (P[j] == 0.0) continue;          /* masked (or underflowed) */
+                    const double *v = V + hoff + (size_t)j * d;
+                    for (int k = 0; k < d; ++k) o[k] += P[j] * v[k];
+                }
+            }
+        free(P);
+    }
+    return err;
+}
+
+/* Backward, recomputing everything from Q, K, V and dO.
+ * Outputs dQ, dK, dV [BH,N,d]; optional O [BH,N,d], LSE [BH,N] and D [BH,N]
+ * (pass NULL to skip).  Pass 1 goes row by row (P_i, D_i, dQ_i, O_i, LSE_i);
+ * pass 2 goes key column by key column (dV_j, dK_j), rebuilding P_ij as
+ * exp(S_ij - LSE_i), the same softmax value written through its normaliser. */
+int oracle_bwd(const double *Q, const double *K, const double *V, const double *dO,
+               int BH, int N, int d, int kind, const uint8_t *block_mask, int block,
+               double scale, double *dQ, double *dK, double *dV,
+               double *O, double *LSE, double *D)
+{
+    spec_t s = make_spec(N, d, kind, block_mask, block, scale);
+    if (check(&s, BH) != OR_OK || !Q || !K || !V || !dO || !dQ || !dK || !dV) return OR_ERR_ARG;
+    double *lse = (double *)malloc(sizeof(double) * (size_t)BH * N);
+    double *Dv = (double *)malloc(sizeof(double) * (size_t)BH * N);
+    if (!lse || !Dv) { free(lse); free(Dv); return OR_ERR_NOMEM; }
+    int err = OR_OK;
+
+    /* pass 1: rows */
+#pragma omp parallel
+    {
+        double *P = (double *)malloc(sizeof(double) * (size_t)N);
+        double *dP = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!P || !dP) {
+#pragma omp atomic write
+            err = OR_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 8) collapse(2)
+        for (int h = 0; h < BH; ++h)
+            for (int i = 0; i < N; ++i) {
+                if (!P || !dP) continue;
+                const size_t hoff = (size_t)h * N * d;
+                const double *dq_o = dO + hoff + (size_t)i * d;
+                double m = score_row(&s, Q + hoff, K + hoff, i, P);
+                double L = softmax_row(&s, P, m);
+                double Di = 0.0;
+                for (int j = 0; j < N; ++j) {
+                    dP[j] = 0.0;
+                    if (P[j] == 0.0) continue;
+                    dP[j] = dot(dq_o, V + hoff + (size_t)j * d, d);
+                    Di += P[j] * dP[j];
+                }
+                double *dq = dQ + hoff + (size_t)i * d;
+                for (int k = 0; k < d; ++k) dq[k] = 0.0;
+                for (int j = 0; j < N; ++j) {
+                    if (P[j] == 0.0) continue;
+                    double ds = P[j] * (dP[j] - Di);
+                    const double *kj = K + hoff + (size_t)j * d;
+                    for (int k = 0; k < d; ++k) dq[k] += ds * kj[k];
+                }
+                for (int k = 0; k < d; ++k) dq[k] *= scale;
+                if (O) {
+                    double *o = O + hoff + (size_t)i * d;
+                    for (int k = 0; k < d; ++k) o[k] = 0.0;
+                    for (int j = 0; j < N; ++j) {
+                        if (P[j] == 0.0) continue;
+                        const double *v = V + hoff + (size_t)j * d;
+                        for (int k = 0; k < d; ++k) o[k] += P[j] * v[k];
+                    }
+                }
+                lse[(size_t)h * N + i] = L;
+                Dv[(size_t)h * N + i] = Di;
+            }
+        free(P);
+        free(dP);
+    }
+
+    /* pass 2: key columns */
+    if (err == OR_OK) {
+#pragma omp parallel for schedule(dynamic, 8) collapse(2)
+        for (int h = 0; h < BH; ++h)
+            for (int j = 0; j < N; ++j) {
+                const size_t hoff = (size_t)h * N * d;
+                const double *kj = K + hoff + (size_t)j * d;
+                const double *vj = V + hoff + (size_t)j * d;
+                double *dk = dK + hoff + (size_t)j * d;
+                double *dv = dV + hoff + (size_t)j * d;
+                for (int k = 0; k < d; ++k) { dk[k] = 0.0; dv[k] = 0.0; }
+                for (int i = 0; i < N; ++i) {
+                    if (!allowed(&s, i, j)) continue;
+                    const double L = lse[(size_t)h * N + i];
+                    if (L == -INFINITY) continue;
+                    const double *qi = Q + hoff + (size_t)i * d;
+                    const double *doi = dO + hoff + (size_t)i * d;
+                    double p = exp(s.scale * dot(qi, kj, d) - L);
+                    double dp = dot(doi, vj, d);
+                    double ds = p * (dp - Dv[(size_t)h * N + i]);
+                    for (int k = 0; k < d; ++k) {
+                        dv[k] += p * doi[k];
+                        dk[k] += ds * qi[k];
+                    }
+                }
+                for (int k = 0; k < d; ++k) dk[k] *= scale;
+            }
+    }
+    if (LSE) memcpy(LSE, lse, sizeof(double) * (size_t)BH * N);
+    if (D) memcpy(D, Dv, sizeof(double) * (size_t)BH * N);
+    free(lse);
+    free(Dv);
+    return err;
+}
+
+/* Selected rows: for each (head[r], row[r]) pair, O_r [d], LSE_r and, when dO
+ * is given, dQ_r [d].  Everything here depends on that one query row only,
+ * so the cost is O(N d) per row whatever the problem size. */
+int oracle_rows(const double *Q, const double *K, const double *V, const double *dO,
+                int BH, int N, int d, int kind, const uint8_t *block_mask, int block,
+                double scale, const int *head, const int *row, int nrows,
+                double *O, double *LSE, double *dQ)
+{
+    spec_t s = make_spec(N, d, kind, block_mask, block, scale);
+    if (check(&s, BH) != OR_OK || !Q || !K || !V || !head || !row || nrows < 0 || !O || !LSE)
+        return OR_ERR_ARG;
+    if (dQ && !dO) return OR_ERR_ARG;
+    for (int r = 0; r < nrows; ++r)
+        if (head[r] < 0 || head[r] >= BH || row[r] < 0 || row[r] >= N) return OR_ERR_ARG;
+    int err = OR_OK;
+#pragma omp parallel
+    {
+        double *P = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!P) {
+#pragma omp atomic write
+            err = OR_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int r = 0; r < nrows; ++r) {
+            if (!P) continue;
+            const size_t hoff = (size_t)head[r] * N * d;
+            const int i = row[r];
+            double m = score_row(&s, Q + hoff, K + hoff, i, P);
+            LSE[r] = softmax_row(&s, P, m);
+            double *o = O + (size_t)r * d;
+            for (int k = 0; k < d; ++k) o[k] = 0.0;
+            for (int j = 0; j < N; ++j) {
+                if (P[j] == 0.0) continue;
+                const double *v = V + hoff + (size_t)j * d;
+                for (int k = 0; k < d; ++k) o[k] += P[j] * v[k];
+            }
+            if (dQ) {
+                const double *doi = dO + hoff + (size_t)i * d;
+                double Di = 0.0;
+                for (int j = 0; j < N; ++j)
+                    if (P[j] != 0.0) Di += P[j] * dot(doi, V + hoff + (size_t)j * d, d);
+                double *dq = dQ + (size_t)r * d;
+                for (int k = 0; k < d; ++k) dq[k] = 0.0;
+                for (int j = 0; j < N; ++j) {
+                    if (P[j] == 0.0) continue;
+                    double ds = P[j] * (dot(doi, V + hoff + (size_t)j * d, d) - Di);
+                    const double *kj = K + hoff + (size_t)j * d;
+                    for (int k = 0; k < d; ++k) dq[k] += ds * kj[k];
+                }
+                for (int k = 0; k < d; ++k) dq[k] *= scale;
+            }
+        }
+        free(P);
+    }
+    return err;
+}
+
+/* Full probability matrix P [BH,N,N] (small N only). */
+int oracle_probs(const double *Q, const double *K, int BH, int N, int d, int kind,
+                 const uint8_t *block_mask, int block, double scale, double *P)
+{
+    spec_t s = make_spec(N, d, kind, block_mask, block, scale);
+    if (check(&s, BH) != OR_OK || !Q || !K || !P) return OR_ERR_ARG;
+#pragma omp parallel for schedule(static) collapse(2)
+    for (int h = 0; h < BH; ++h)
+        for (int i = 0; i < N; ++i) {
+            const size_t hoff = (size_t)h * N * d;
+            double *Prow = P + ((size_t)h * N + i) * N;
+            double m = score_row(&s, Q + hoff, K + hoff, i, Prow);
+            softmax_row(&s, Prow, m);
+        }
+    return OR_OK;
+}
