@@ -1,0 +1,152 @@
+"""Exact IO-aware attention (FlashAttention forward and backward) for B200.
+
+A thin ctypes binding over ``libfa.so``: it only checks tensor properties and
+marshals pointers, sizes and the CUDA stream into the C ABI declared in
+``include/fa.h``.  Every step of the computation runs in the library's CUDA
+kernels; there is no fallback path.  PyTorch supplies device memory and
+streams.
+
+    O, LSE = fa.fwd(Q, K, V, mask="causal", scale=d ** -0.5)
+    dQ, dK, dV = fa.bwd(Q, K, V, O, dO, LSE, mask="causal", scale=d ** -0.5)
+
+Tensors are bf16 [B, H, N, d] contiguous CUDA tensors, LSE is fp32 [B, H, N].
+``block_mask`` (mask="block") is a uint8 [ceil(N/128), ceil(N/128)] CUDA
+tensor shared by every batch and head.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+MASKS = {"none": 0, "causal": 1, "block": 2}
+STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
+          4: "FA_ERR_WORKSPACE", 5: "FA_ERR_TIMEOUT"}
+
+# Every symbol include/fa.h declares, with its ctypes signature.
+_vp, _i, _f, _sz, _u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
+SIGNATURES = {
+    "fa_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp]),
+    "fa_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "fa_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "fa_device_status": (_i, [_vp]),
+    "fa_set_wait_timeout_ns": (None, [_u64]),
+    "fa_status_string": (ctypes.c_char_p, [_i]),
+    "fa_selftest_bounded_wait": (_i, [_u64, _vp]),
+    "fa_selftest_mma_tile": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
+}
+
+
+class FAError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfa.so (build it first with ``python -m exact_io_aware_65_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise FAError(3, f"CUDA library missing at {LIB_PATH}; build it with "
+                             "`python -m exact_io_aware_65_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise FAError(code, what)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _mask(mask, block_mask):
+    kind = MASKS[mask] if isinstance(mask, str) else int(mask)
+    ptr = None
+    if kind == MASKS["block"]:
+        if block_mask is None or not block_mask.is_cuda or block_mask.dtype != torch.uint8:
+            raise FAError(1, "block mask must be a uint8 CUDA tensor")
+        ptr = block_mask.contiguous().data_ptr()
+    return kind, ptr
+
+
+def _check_qkv(*ts):
+    for t in ts:
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
+            raise FAError(1, "tensors must be contiguous bf16 CUDA tensors [B, H, N, d]")
+
+
+def fwd(Q, K, V, mask="none", block_mask=None, scale=None, O=None, LSE=None, stream=None):
+    """O [B,H,N,d] bf16 and LSE [B,H,N] fp32 (natural log)."""
+    _check_qkv(Q, K, V)
+    B, H, N, d = Q.shape
+    scale = d ** -0.5 if scale is None else float(scale)
+    kind, mptr = _mask(mask, block_mask)
+    if O is None:
+        O = torch.empty_like(Q)
+    if LSE is None:
+        LSE = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    _check(lib().fa_fwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, H, N, d, kind, mptr, scale,
+                        O.data_ptr(), LSE.data_ptr(), _stream(stream)), "fa_fwd")
+    return O, LSE
+
+
+def bwd_workspace_size(B, H, N, d) -> int:
+    return int(lib().fa_bwd_workspace_size(B, H, N, d))
+
+
+def bwd(Q, K, V, O, dO, LSE, mask="none", block_mask=None, scale=None, dQ=None, dK=None, dV=None,
+        workspace=None, stream=None):
+    """dQ, dK, dV [B,H,N,d] bf16."""
+    _check_qkv(Q, K, V, O, dO)
+    B, H, N, d = Q.shape
+    scale = d ** -0.5 if scale is None else float(scale)
+    kind, mptr = _mask(mask, block_mask)
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(V) if dV is None else dV
+    ws = bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=Q.device)
+    _check(lib().fa_bwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(), dO.data_ptr(),
+                        LSE.data_ptr(), B, H, N, d, kind, mptr, scale, dQ.data_ptr(), dK.data_ptr(),
+                        dV.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)),
+           "fa_bwd")
+    return dQ, dK, dV
+
+
+def device_status(stream=None) -> int:
+    """Synchronise and read/clear the device status word (0 = ok, 5 = timeout)."""
+    return int(lib().fa_device_status(_stream(stream)))
+
+
+def set_wait_timeout_ns(ns: int):
+    lib().fa_set_wait_timeout_ns(int(ns))
+
+
+def selftest_bounded_wait(timeout_ns: int, stream=None):
+    _check(lib().fa_selftest_bounded_wait(int(timeout_ns), _stream(stream)), "fa_selftest_bounded_wait")
+
+
+def selftest_mma_tile(A, B, n, k, mode, stream=None):
+    C = torch.empty((128, n), dtype=torch.float32, device=A.device)
+    _check(lib().fa_selftest_mma_tile(A.data_ptr(), B.data_ptr(), C.data_ptr(), n, k, mode, _stream(stream)),
+           "fa_selftest_mma_tile")
+    return C

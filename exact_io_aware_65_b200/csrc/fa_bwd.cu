@@ -1,0 +1,617 @@
+// fa_bwd.cu -- backward pass of exact attention on sm_100a.
+//
+// The pages fix the strategy ("FlashAttention: Fast and Memory-Efficient
+// Exact Attention with IO-Awareness", section "Backward / recomputation"):
+// the forward keeps only the per-row softmax statistic (here LSE), and the
+// backward rebuilds the attention probabilities on chip instead of reading an
+// N x N matrix back.  The gradient formulas are the calculus of softmax
+// attention:
+//     P_ij  = exp(scale q_i.k_j - LSE_i)           (recomputed)
+//     dV_j  = sum_i P_ij dO_i
+//     dP_ij = dO_i . v_j,   D_i = dO_i . O_i = sum_j P_ij dP_ij
+//     dS_ij = P_ij (dP_ij - D_i)
+//     dK_j  = scale sum_i dS_ij q_i,   dQ_i = scale sum_j dS_ij k_j
+//
+// Three kernels, all on the caller's stream:
+//   prep     D_i, LSE_i * log2(e) (padded to whole tiles) and a zeroed fp32
+//            dQ accumulator, in the workspace.
+//   main     one persistent CTA per SM; a work item is one (head, 128-key
+//            tile).  K_j and V_j stay in shared memory, dK_j and dV_j
+//            accumulate in tensor memory across the query tiles that see
+//            them, so they need no atomics.  Per query tile:
+//              S^T  = K_j Q_i^T,  dP^T = V_j dO_i^T        (tensor cores)
+//              P^T, dS^T                                   (softmax warps)
+//              dV  += P^T dO_i,   dK += dS^T Q_i            (A from tensor memory)
+//              dQ_i = dS K_j                                 (A = dS^T in smem)
+//            and dQ_i is added to the fp32 accumulator with vector
+//            reductions by four drain warps.
+//   convert  dQ = bf16(scale * dQ_acc).
+//
+// CTA roles (512 threads): warp 0 TMA producer; warp 1 MMA issuer; warps
+// 4..11 softmax (thread = key row; warps 4..7 take query columns 0..63,
+// warps 8..11 columns 64..127); warps 12..15 dQ drain (thread = query row).
+// Tensor memory: S^T [0,128) then P^T (bf16) in [0,64); dP^T [128,256) then
+// dS^T (bf16) in [128,192); dV [256, 256+d); dK [256+d, 256+2d).  The dQ
+// tile sits in the columns P and dS left free ([64,128) and [192,256)) for
+// d = 128, and in two buffers at [384,448) and [448,512) for d = 64.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace bwd {
+
+constexpr int BK = 128;  // keys per work item
+constexpr int BQ = 128;  // queries per step
+constexpr int NUM_THREADS = 512;
+constexpr float LOG2E = 1.4426950408889634074f;
+
+__host__ __device__ constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace carve-up (all offsets 256-byte aligned).
+struct Workspace {
+  size_t dq_off, d_off, l2_off, total;
+};
+__host__ __device__ inline Workspace workspace_layout(int BH, int Npad, int d) {
+  Workspace w;
+  w.dq_off = 0;
+  w.d_off = align256((size_t)BH * Npad * d * sizeof(float));
+  w.l2_off = w.d_off + align256((size_t)BH * Npad * sizeof(float));
+  w.total = w.l2_off + align256((size_t)BH * Npad * sizeof(float));
+  return w;
+}
+
+// ------------------------------------------------------------------ prep ---
+// One group of d/8 lanes per row; each lane covers 8 elements (16 bytes).
+template <int D>
+__global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restrict__ O,
+                                                   const __nv_bfloat16* __restrict__ dO,
+                                                   const float* __restrict__ LSE, float* __restrict__ Dw,
+                                                   float* __restrict__ L2w, float* __restrict__ dq_acc, int BH, int N,
+                                                   int Npad) {
+  constexpr int LPR = D / 8;
+  constexpr int RPW = 32 / LPR;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPR, li = lane % LPR;
+  const long long total = (long long)BH * Npad;
+  const long long warps = (long long)gridDim.x * (blockDim.x / 32);
+  for (long long r0 = ((long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)) * RPW; r0 < total;
+       r0 += warps * RPW) {
+    const long long r = r0 + sub;
+    const int bh = (int)(r / Npad), n = (int)(r % Npad);
+    const bool real = r < total && n < N;
+    float acc = 0.0f;
+    if (real) {
+      const size_t e = ((size_t)bh * N + n) * D + li * 8;
+      const uint4 a = *reinterpret_cast<const uint4*>(O + e);
+      const uint4 b = *reinterpret_cast<const uint4*>(dO + e);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 fa2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[i]));
+        const float2 fb2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[i]));
+        acc = fmaf(fa2.x, fb2.x, acc);
+        acc = fmaf(fa2.y, fb2.y, acc);
+      }
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (r < total) {
+      if (li == 0) {
+        Dw[r] = acc;
+        float l2 = INFINITY;  // padding rows and rows that saw no key: P = 0
+        if (real) {
+          const float lse = LSE[(size_t)bh * N + n];
+          if (lse > -INFINITY) l2 = lse * LOG2E;
+        }
+        L2w[r] = l2;
+      }
+      float4* z = reinterpret_cast<float4*>(dq_acc + (size_t)r * D + li * 8);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+}
+
+// --------------------------------------------------------------- convert ---
+template <int D>
+__global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict__ dq_acc,
+                                                         __nv_bfloat16* __restrict__ dQ, int BH, int N, int Npad,
+                                                         float scale) {
+  const long long total = (long long)BH * N * (D / 8);
+  for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < total;
+       g += (long long)gridDim.x * blockDim.x) {
+    const long long row = g / (D / 8);
+    const int c8 = (int)(g % (D / 8)) * 8;
+    const int bh = (int)(row / N), n = (int)(row % N);
+    const float4* s = reinterpret_cast<const float4*>(dq_acc + ((size_t)bh * Npad + n) * D + c8);
+    const float4 a = s[0], b = s[1];
+    uint4 o;
+    o.x = pack_bf16x2(a.x * scale, a.y * scale);
+    o.y = pack_bf16x2(a.z * scale, a.w * scale);
+    o.z = pack_bf16x2(b.x * scale, b.y * scale);
+    o.w = pack_bf16x2(b.z * scale, b.w * scale);
+    *reinterpret_cast<uint4*>(dQ + (size_t)row * D + c8) = o;
+  }
+}
+
+// ------------------------------------------------------------------ main ---
+template <int D>
+struct Cfg {
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int CHUNKS = D / 64;
+  static constexpr int CHUNK_BYTES = 128 * 128;  // 128 rows x 128 bytes
+  static constexpr int NST = D == 64 ? 4 : 2;    // Q/dO stages
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = TILE_BYTES;
+  static constexpr int OFF_DS = 2 * TILE_BYTES;           // dS^T, 128 x 128 bf16 (2 chunks)
+  static constexpr int OFF_QD = 2 * TILE_BYTES + 32768;   // stages of (Q, dO)
+  static constexpr int SMEM_BYTES = OFF_QD + NST * 2 * TILE_BYTES + 1024;
+  static constexpr int COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
+  static constexpr int NDQ = D == 64 ? 2 : 1;  // dQ buffers in tensor memory
+};
+
+struct Params {
+  int BH, N, Npad, nq, n_items, mask_kind;
+  const uint8_t* block_mask;
+  float scale, scale_log2;
+  const float* Dw;
+  const float* L2w;
+  float* dq_acc;
+  __nv_bfloat16* dK;
+  __nv_bfloat16* dV;
+  uint64_t timeout_ns;
+  uint32_t* status;
+};
+
+struct Item {
+  int bh, j;
+};
+
+// Work item idx -> (head, key tile); low key tiles first: under a causal
+// mask they meet the most query tiles.
+__device__ __forceinline__ Item item_at(const Params& p, int idx) {
+  Item it;
+  it.j = idx / p.BH;
+  it.bh = idx % p.BH;
+  return it;
+}
+
+// Next query tile >= i that attends to key tile j (nq if none).
+__device__ __forceinline__ int next_q(const Params& p, int j, int i) {
+  if (p.mask_kind == FA_MASK_CAUSAL) return i < j ? j : i;
+  if (p.mask_kind == FA_MASK_BLOCK) {
+    for (; i < p.nq; ++i)
+      if (__ldg(p.block_mask + (size_t)i * p.nq + j)) return i;
+  }
+  return i;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapdO,
+                const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  __shared__ __align__(8) uint64_t kv_full, kv_empty, s_full, p_full, ds_full, dkdv_full, mma_drain;
+  __shared__ __align__(8) uint64_t qd_full[C::NST], qd_empty[C::NST], dq_full[C::NDQ], dq_free[C::NDQ];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&kv_full, 1);
+    mbar_init(&kv_empty, 1);
+    mbar_init(&s_full, 1);
+    mbar_init(&p_full, 256);
+    mbar_init(&ds_full, 256);
+    mbar_init(&dkdv_full, 1);
+    mbar_init(&mma_drain, 1);
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(&qd_full[s], 1);
+      mbar_init(&qd_empty[s], 1);
+    }
+    for (int b = 0; b < C::NDQ; ++b) {
+      mbar_init(&dq_full[b], 1);
+      mbar_init(&dq_free[b], 128);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapQ);
+    tma_prefetch_desc(&mapK);
+    tma_prefetch_desc(&mapV);
+    tma_prefetch_desc(&mapdO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const WaitCtx w{p.timeout_ns, &abort_flag, p.status};
+
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  uint8_t* sDS = smem + C::OFF_DS;
+  uint8_t* sQD = smem + C::OFF_QD;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t item_iter = 0, qd_iter = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_iter) {
+        const Item it = item_at(p, idx);
+        ok = mbar_wait(&kv_empty, (item_iter & 1) ^ 1, w);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&kv_full, 2 * C::TILE_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::CHUNKS; ++c) {
+          tma_load_3d(sK + c * C::CHUNK_BYTES, &mapK, &kv_full, c * 64, it.j * BK, it.bh);
+          tma_load_3d(sV + c * C::CHUNK_BYTES, &mapV, &kv_full, c * 64, it.j * BK, it.bh);
+        }
+        for (int i = next_q(p, it.j, 0); i < p.nq; i = next_q(p, it.j, i + 1)) {
+          const uint32_t st = qd_iter % C::NST;
+          ok = mbar_wait(&qd_empty[st], ((qd_iter / C::NST) & 1) ^ 1, w);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&qd_full[st], 2 * C::TILE_BYTES);
+          uint8_t* q = sQD + st * 2 * C::TILE_BYTES;
+#pragma unroll
+          for (int c = 0; c < C::CHUNKS; ++c) {
+            tma_load_3d(q + c * C::CHUNK_BYTES, &mapQ, &qd_full[st], c * 64, i * BQ, it.bh);
+            tma_load_3d(q + C::TILE_BYTES + c * C::CHUNK_BYTES, &mapdO, &qd_full[st], c * 64, i * BQ, it.bh);
+          }
+          ++qd_iter;
+        }
+      }
+      if (!ok) {
+        const uint64_t dl = globaltimer_ns() + 100000000ull;
+        const uint32_t n = qd_iter < (uint32_t)C::NST ? qd_iter : (uint32_t)C::NST;
+        for (uint32_t k = 0; k < n; ++k) {
+          const uint32_t q = qd_iter - 1 - k;
+          mbar_drain_wait(&qd_full[q % C::NST], (q / C::NST) & 1, dl);
+        }
+        if (item_iter > 0) mbar_drain_wait(&kv_full, (item_iter - 1) & 1, dl);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_T = idesc_bf16_f32(128, 128, 0, 0);   // S^T, dP^T: K-major A and B
+      constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, 0, 1);     // dV, dK: A in TMEM, B MN-major
+      constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, 64, 1, 1);    // dQ (64-column pieces): both MN-major
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aDS = smem_u32(sDS), aQD = smem_u32(sQD);
+      uint32_t item_iter = 0, qd_iter = 0, dq_iter = 0, p_cnt = 0, ds_cnt = 0;
+      bool ok = true, issued = false;
+      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_iter) {
+        const Item it = item_at(p, idx);
+        ok = mbar_wait(&kv_full, item_iter & 1, w);
+        if (!ok) break;
+        int n = 0;
+        for (int i = next_q(p, it.j, 0); ok && i < p.nq; i = next_q(p, it.j, i + 1), ++n) {
+          const uint32_t st = qd_iter % C::NST;
+          const uint32_t b = dq_iter % C::NDQ;
+          ok = mbar_wait(&qd_full[st], (qd_iter / C::NST) & 1, w);
+          // The dQ buffer about to be written must have been drained.  For
+          // d = 128 it overlaps the S^T / dP^T columns, so wait before those.
+          if (ok && dq_iter >= (uint32_t)C::NDQ) ok = mbar_wait(&dq_free[b], ((dq_iter / C::NDQ) - 1) & 1, w);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t aQ = aQD + st * 2 * C::TILE_BYTES;
+          const uint32_t adO = aQ + C::TILE_BYTES;
+          // S^T = K Q^T and dP^T = V dO^T (M = keys, N = queries, K = d)
+#pragma unroll
+          for (int s = 0; s < D / 16; ++s) {
+            const uint32_t off = (s >> 2) * C::CHUNK_BYTES + (s & 3) * 32;
+            mma_ss(tmem + C::COL_S, smem_desc_sw128(aK + off, 16, 1024), smem_desc_sw128(aQ + off, 16, 1024),
+                   IDESC_T, s > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int s = 0; s < D / 16; ++s) {
+            const uint32_t off = (s >> 2) * C::CHUNK_BYTES + (s & 3) * 32;
+            mma_ss(tmem + C::COL_DP, smem_desc_sw128(aV + off, 16, 1024), smem_desc_sw128(adO + off, 16, 1024),
+                   IDESC_T, s > 0 ? 1u : 0u);
+          }
+          tc_commit(&s_full);
+          issued = true;
+          // dV += P^T dO (A = P^T in TMEM, K = 128 queries)
+          ok = mbar_wait(&p_full, p_cnt & 1, w);
+          if (!ok) break;
+          ++p_cnt;
+          tc_fence_after();
+#pragma unroll
+          for (int s = 0; s < BQ / 16; ++s)
+            mma_ts(tmem + C::COL_DV, tmem + C::COL_S + s * 8, smem_desc_sw128(adO + s * 2048, C::CHUNK_BYTES, 1024),
+                   IDESC_G, (n > 0 || s > 0) ? 1u : 0u);
+          // dK += dS^T Q; dQ_i = dS K
+          ok = mbar_wait(&ds_full, ds_cnt & 1, w);
+          if (!ok) break;
+          ++ds_cnt;
+          tc_fence_after();
+#pragma unroll
+          for (int s = 0; s < BQ / 16; ++s)
+            mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + s * 8, smem_desc_sw128(aQ + s * 2048, C::CHUNK_BYTES, 1024),
+                   IDESC_G, (n > 0 || s > 0) ? 1u : 0u);
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h) {
+            const uint32_t col = D == 128 ? (h == 0 ? 64u : 192u) : (384u + 64u * b);
+#pragma unroll
+            for (int s = 0; s < BK / 16; ++s)
+              mma_ss(tmem + col, smem_desc_sw128(aDS + s * 2048, C::CHUNK_BYTES, 1024),
+                     smem_desc_sw128(aK + h * C::CHUNK_BYTES + s * 2048, C::CHUNK_BYTES, 1024), IDESC_Q,
+                     s > 0 ? 1u : 0u);
+          }
+          tc_commit(&dq_full[b]);
+          tc_commit(&qd_empty[st]);
+          ++qd_iter;
+          ++dq_iter;
+        }
+        if (!ok) break;
+        tc_commit(&dkdv_full);
+        tc_commit(&kv_empty);
+      }
+      if (issued) {
+        tc_commit(&mma_drain);
+        mbar_drain_wait(&mma_drain, 0, globaltimer_ns() + 100000000ull);
+      }
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------------------ softmax
+    const int quarter = warp & 3;
+    const int hf = (warp - 4) >> 2;        // query half: columns [64 hf, 64 hf + 64)
+    const int kr = quarter * 32 + lane;    // key row within the tile
+    const uint32_t lane_bits = uint32_t(quarter * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint32_t s_cnt = 0, dk_cnt = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x) {
+      const Item it = item_at(p, idx);
+      const int key = it.j * BK + kr;
+      bool any = false;
+      for (int i = next_q(p, it.j, 0); i < p.nq; i = next_q(p, it.j, i + 1)) {
+        ok = mbar_wait_warp(&s_full, s_cnt & 1, w);
+        if (!ok) break;
+        ++s_cnt;
+        tc_fence_after();
+        const int q0 = i * BQ + hf * 64;  // first query of this thread's half
+        const size_t rowbase = (size_t)it.bh * p.Npad + q0;
+        const bool key_live = key < p.N;
+        const bool diag = p.mask_kind == FA_MASK_CAUSAL && i == it.j;
+        float pr[64];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t sr[32];
+          FA_TMEM_LD_X32(tmem + lane_bits + C::COL_S + hf * 64 + cc * 32, sr);
+          tc_wait_ld();
+          const float4* l4 = reinterpret_cast<const float4*>(p.L2w + rowbase + cc * 32);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float4 lv = __ldg(l4 + u);
+            const float lvv[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int col = cc * 32 + u * 4 + e;
+              float pv = ex2_approx(fmaf(__uint_as_float(sr[u * 4 + e]), sl2, -lvv[e]));
+              if (!key_live || (diag && hf * 64 + col < kr)) pv = 0.0f;
+              pr[col] = pv;
+            }
+          }
+        }
+        {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
+          FA_TMEM_ST_X32(tmem + lane_bits + C::COL_S + hf * 32, pk);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full);
+        // dS^T = P^T * (dP^T - D)
+        uint8_t* ds_chunk = sDS + hf * C::CHUNK_BYTES + kr * 128;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t dr[32];
+          FA_TMEM_LD_X32(tmem + lane_bits + C::COL_DP + hf * 64 + cc * 32, dr);
+          tc_wait_ld();
+          const float4* d4 = reinterpret_cast<const float4*>(p.Dw + rowbase + cc * 32);
+          uint32_t pk[16];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float4 dv = __ldg(d4 + u);
+            const int c = cc * 32 + u * 4;
+            const float g0 = pr[c + 0] * (__uint_as_float(dr[u * 4 + 0]) - dv.x);
+            const float g1 = pr[c + 1] * (__uint_as_float(dr[u * 4 + 1]) - dv.y);
+            const float g2 = pr[c + 2] * (__uint_as_float(dr[u * 4 + 2]) - dv.z);
+            const float g3 = pr[c + 3] * (__uint_as_float(dr[u * 4 + 3]) - dv.w);
+            pk[u * 2 + 0] = pack_bf16x2(g0, g1);
+            pk[u * 2 + 1] = pack_bf16x2(g2, g3);
+          }
+          FA_TMEM_ST_X16(tmem + lane_bits + C::COL_DP + hf * 32 + cc * 16, pk);
+          // shared-memory copy, 128-byte swizzle: 16-byte unit u of row kr
+          // lives at unit (u ^ (kr & 7)).
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int unit = (cc * 4 + u) ^ (kr & 7);
+            *reinterpret_cast<uint4*>(ds_chunk + unit * 16) =
+                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          }
+        }
+        tc_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&ds_full);
+        any = true;
+      }
+      if (!ok) break;
+      // ---- epilogue: dV and dK rows of this key tile
+      ok = mbar_wait_warp(&dkdv_full, dk_cnt & 1, w);
+      if (!ok) break;
+      ++dk_cnt;
+      tc_fence_after();
+      const bool store = key < p.N;
+      const size_t gbase = ((size_t)it.bh * p.N + key) * D;
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {  // 0: dV, 1: dK
+        const float mul = g == 0 ? 1.0f : p.scale;
+        __nv_bfloat16* dst = (g == 0 ? p.dV : p.dK) + gbase;
+        const int colbase = (g == 0 ? C::COL_DV : C::COL_DK) + hf * (D / 2);
+#pragma unroll
+        for (int c = 0; c < D / 2; c += 32) {
+          uint32_t v[32];
+          FA_TMEM_LD_X32(tmem + lane_bits + colbase + c, v);
+          tc_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = any ? pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul) : 0u;
+          if (store) {
+            uint4* o = reinterpret_cast<uint4*>(dst + hf * (D / 2) + c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+    }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ dQ drain
+    const int quarter = warp & 3;
+    const int qr = quarter * 32 + lane;
+    const uint32_t lane_bits = uint32_t(quarter * 32) << 16;
+    uint32_t dq_iter = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x) {
+      const Item it = item_at(p, idx);
+      for (int i = next_q(p, it.j, 0); i < p.nq; i = next_q(p, it.j, i + 1)) {
+        const uint32_t b = dq_iter % C::NDQ;
+        ok = mbar_wait_warp(&dq_full[b], (dq_iter / C::NDQ) & 1, w);
+        if (!ok) break;
+        tc_fence_after();
+        float* dst = p.dq_acc + ((size_t)it.bh * p.Npad + (size_t)i * BQ + qr) * D;
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+          const uint32_t col = D == 128 ? (h == 0 ? 64u : 192u) : (384u + 64u * b);
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t v[32];
+            FA_TMEM_LD_X32(tmem + lane_bits + col + cc * 32, v);
+            tc_wait_ld();
+            float* d = dst + h * 64 + cc * 32;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              red_add_v4(d + 4 * e, __uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                         __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&dq_free[b]);
+        ++dq_iter;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace bwd
+
+size_t bwd_workspace_bytes(int B, int H, int N, int d) {
+  const int Npad = ((N + 127) / 128) * 128;
+  return bwd::workspace_layout(B * H, Npad, d).total;
+}
+
+template <int D>
+static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CUtensorMap& mK, const CUtensorMap& mV,
+                              const CUtensorMap& mdO, const void* O, const void* dO, const float* LSE, void* dQ,
+                              void* dK, void* dV, void* workspace, cudaStream_t s, uint32_t* st) {
+  const int Npad = pr.nq * 128;
+  const bwd::Workspace wl = bwd::workspace_layout(pr.BH, Npad, D);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(ws + wl.dq_off);
+  float* Dw = reinterpret_cast<float*>(ws + wl.d_off);
+  float* L2w = reinterpret_cast<float*>(ws + wl.l2_off);
+  const int sms = num_sms();
+
+  {
+    const long long rows = (long long)pr.BH * Npad;
+    const long long warps_needed = (rows + (32 / (D / 8)) - 1) / (32 / (D / 8));
+    long long blocks = (warps_needed + 7) / 8;
+    if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
+    bwd::prep_kernel<D><<<(int)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(O),
+                                                     static_cast<const __nv_bfloat16*>(dO), LSE, Dw, L2w, dq_acc,
+                                                     pr.BH, pr.N, Npad);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  {
+    bwd::Params p;
+    p.BH = pr.BH;
+    p.N = pr.N;
+    p.Npad = Npad;
+    p.nq = pr.nq;
+    p.n_items = pr.BH * pr.nq;
+    p.mask_kind = pr.mask_kind;
+    p.block_mask = pr.block_mask;
+    p.scale = pr.scale;
+    p.scale_log2 = pr.scale_log2;
+    p.Dw = Dw;
+    p.L2w = L2w;
+    p.dq_acc = dq_acc;
+    p.dK = static_cast<__nv_bfloat16*>(dK);
+    p.dV = static_cast<__nv_bfloat16*>(dV);
+    p.timeout_ns = wait_timeout_ns();
+    p.status = st;
+    constexpr int smem = bwd::Cfg<D>::SMEM_BYTES;
+    if (cudaFuncSetAttribute(bwd::main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return FA_ERR_CUDA;
+    const int grid = p.n_items < sms ? p.n_items : sms;
+    bwd::main_kernel<D><<<grid, bwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, mdO, p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  {
+    const long long work = (long long)pr.BH * pr.N * (D / 8);
+    long long blocks = (work + 255) / 256;
+    if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
+    bwd::dq_convert_kernel<D><<<(int)blocks, 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), pr.BH, pr.N,
+                                                          Npad, pr.scale);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+fa_status launch_bwd(const Problem& pr, const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                     const float* LSE, void* dQ, void* dK, void* dV, void* workspace, cudaStream_t s) {
+  uint32_t* st = status_word();
+  if (!st) return FA_ERR_CUDA;
+  CUtensorMap mQ, mK, mV, mdO;
+  if (!make_map_bf16(&mQ, Q, pr.BH, pr.N, pr.d, 128) || !make_map_bf16(&mK, K, pr.BH, pr.N, pr.d, 128) ||
+      !make_map_bf16(&mV, V, pr.BH, pr.N, pr.d, 128) || !make_map_bf16(&mdO, dO, pr.BH, pr.N, pr.d, 128))
+    return FA_ERR_CUDA;
+  if (pr.d == 64) return launch_bwd_d<64>(pr, mQ, mK, mV, mdO, O, dO, LSE, dQ, dK, dV, workspace, s, st);
+  return launch_bwd_d<128>(pr, mQ, mK, mV, mdO, O, dO, LSE, dQ, dK, dV, workspace, s, st);
+}
+
+}  // namespace fa

@@ -1,0 +1,462 @@
+// fa_fwd.cu -- forward pass of exact attention on sm_100a.
+//
+// The method ("FlashAttention: making attention fast by respecting the memory
+// hierarchy", tiling paragraph; "FlashAttention: Fast and Memory-Efficient
+// Exact Attention with IO-Awareness", sections "Softmax / tiling" and
+// "Implementation"): load a block of queries, stream blocks of keys and
+// values past it, and keep a running row maximum and row sum so that the
+// softmax is completed incrementally; the N x N scores live only on chip.
+//
+// B200 mapping (one persistent CTA per SM, 384 threads):
+//   warp 0        TMA producer: two 128-row Q tiles per work item, then a ring
+//                 of K and V tiles (128 keys x d, 128-byte swizzle).
+//   warp 1        MMA issuer (one thread): S_t = Q_t K_j^T into tensor memory
+//                 (fp32), and O_t += P_t V_j with P_t read from tensor memory.
+//   warps 4..7    softmax for query tile 0; warps 8..11 for query tile 1.
+//                 Thread r owns query row r: it reads its score row from
+//                 tensor memory, keeps the row max m and row sum l in
+//                 registers, writes P (bf16) back over the scores, and does
+//                 the final O / l and LSE epilogue.
+// Tensor memory (512 columns): S/P of tile t at [128 t, 128 t + 128), O of
+// tile t at [256 + d t, 256 + d t + d).
+//
+// The two query tiles ping-pong: while one softmax group works on its scores
+// the tensor cores run the other tile's PV and next QK^T products.
+//
+// The O rescale is lazy: the reference maximum used for exponentials only
+// moves when the true maximum has grown by more than 2^8; l and O always use
+// the same reference, so the final O / l is unchanged (exact in exact
+// arithmetic) while most tiles skip the tensor-memory round trip.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace fwd {
+
+constexpr int BM = 128;              // query rows per tile
+constexpr int BN = 128;              // keys per tile
+constexpr int NUM_THREADS = 384;
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+constexpr float LN2 = 0.69314718055994530942f;
+
+template <int D>
+struct Cfg {
+  static constexpr int TILE_BYTES = BN * D * 2;  // one Q, K or V tile
+  static constexpr int CHUNKS = D / 64;          // 64-column (128-byte) chunks per row
+  static constexpr int CHUNK_BYTES = BN * 128;   // one chunk of a tile
+  static constexpr int NSLOT = D == 64 ? 8 : 4;  // K/V ring slots
+  static constexpr int SMEM_BYTES = 2 * TILE_BYTES + NSLOT * TILE_BYTES + 1024;
+};
+
+struct Params {
+  int BH, N, nq, n_pairs, n_items, mask_kind;
+  const uint8_t* block_mask;
+  float scale_log2;
+  __nv_bfloat16* O;
+  float* LSE;
+  uint64_t timeout_ns;
+  uint32_t* status;
+};
+
+struct Item {
+  int bh, q0, q1;
+  bool has1;
+};
+
+// Work item idx -> (head, pair of query tiles).  Later query tiles come first
+// so that, under a causal mask, the longest items start earliest.
+__device__ __forceinline__ Item item_at(const Params& p, int idx) {
+  Item it;
+  const int c = p.n_pairs - 1 - idx / p.BH;
+  it.bh = idx % p.BH;
+  it.q0 = 2 * c;
+  it.q1 = 2 * c + 1;
+  it.has1 = it.q1 < p.nq;
+  return it;
+}
+
+// Does query tile qt attend to key tile j?
+__device__ __forceinline__ bool member(const Params& p, int qt, int j) {
+  if (p.mask_kind == FA_MASK_CAUSAL) return j <= qt;
+  if (p.mask_kind == FA_MASK_BLOCK) return __ldg(p.block_mask + (size_t)qt * p.nq + j) != 0;
+  return true;
+}
+
+__device__ __forceinline__ int kv_end(const Params& p, const Item& it) {
+  if (p.mask_kind == FA_MASK_CAUSAL) return (it.has1 ? it.q1 : it.q0) + 1;
+  return p.nq;
+}
+
+// Next key tile >= j needed by either query tile of the item (kv_end if none).
+__device__ __forceinline__ int next_union(const Params& p, const Item& it, int j) {
+  const int e = kv_end(p, it);
+  if (p.mask_kind != FA_MASK_BLOCK) return j < e ? j : e;
+  for (; j < e; ++j)
+    if (member(p, it.q0, j) || (it.has1 && member(p, it.q1, j))) return j;
+  return e;
+}
+
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+               const __grid_constant__ CUtensorMap mapV, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;                        // 2 tiles
+  uint8_t* sKV = smem + 2 * C::TILE_BYTES;   // NSLOT tiles
+
+  __shared__ __align__(8) uint64_t q_full, q_empty, mma_drain;
+  __shared__ __align__(8) uint64_t kv_full[C::NSLOT], kv_empty[C::NSLOT];
+  __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_full[2];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int warp = warp_id(), lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&q_full, 1);
+    mbar_init(&q_empty, 1);
+    mbar_init(&mma_drain, 1);
+    for (int i = 0; i < C::NSLOT; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], BM);
+      mbar_init(&o_full[t], 1);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapQ);
+    tma_prefetch_desc(&mapK);
+    tma_prefetch_desc(&mapV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = tmem_base_sh;
+  const WaitCtx w{p.timeout_ns, &abort_flag, p.status};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t kv_iter = 0, item_iter = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_iter) {
+        const Item it = item_at(p, idx);
+        ok = mbar_wait(&q_empty, (item_iter & 1) ^ 1, w);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&q_full, C::TILE_BYTES * (it.has1 ? 2 : 1));
+#pragma unroll
+        for (int c = 0; c < C::CHUNKS; ++c)
+          tma_load_3d(sQ + c * C::CHUNK_BYTES, &mapQ, &q_full, c * 64, it.q0 * BM, it.bh);
+        if (it.has1) {
+#pragma unroll
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_3d(sQ + C::TILE_BYTES + c * C::CHUNK_BYTES, &mapQ, &q_full, c * 64, it.q1 * BM, it.bh);
+        }
+        const int e = kv_end(p, it);
+        for (int j = next_union(p, it, 0); ok && j < e; j = next_union(p, it, j + 1)) {
+          for (int kv = 0; kv < 2; ++kv) {
+            const uint32_t slot = kv_iter % C::NSLOT;
+            ok = mbar_wait(&kv_empty[slot], ((kv_iter / C::NSLOT) & 1) ^ 1, w);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&kv_full[slot], C::TILE_BYTES);
+            uint8_t* dst = sKV + slot * C::TILE_BYTES;
+            const CUtensorMap* m = kv == 0 ? &mapK : &mapV;
+#pragma unroll
+            for (int c = 0; c < C::CHUNKS; ++c)
+              tma_load_3d(dst + c * C::CHUNK_BYTES, m, &kv_full[slot], c * 64, j * BN, it.bh);
+            ++kv_iter;
+          }
+        }
+      }
+      if (!ok) {
+        // Let the loads already issued land before the CTA's shared memory
+        // is released (bounded).
+        const uint64_t dl = globaltimer_ns() + 100000000ull;
+        const uint32_t n = kv_iter < (uint32_t)C::NSLOT ? kv_iter : (uint32_t)C::NSLOT;
+        for (uint32_t i = 0; i < n; ++i) {
+          const uint32_t k = kv_iter - 1 - i;
+          mbar_drain_wait(&kv_full[k % C::NSLOT], (k / C::NSLOT) & 1, dl);
+        }
+        if (item_iter > 0) mbar_drain_wait(&q_full, (item_iter - 1) & 1, dl);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0, 0);
+      constexpr uint32_t IDESC_O = idesc_bf16_f32(BM, D, 0, 1);
+      const uint32_t sQ_addr = smem_u32(sQ);
+      const uint32_t sKV_addr = smem_u32(sKV);
+      uint32_t kv_iter = 0, item_iter = 0, p_cnt[2] = {0, 0};
+      bool ok = true, issued = false;
+
+      auto issue_s = [&](int t, uint32_t kslot) {
+        const uint32_t qa = sQ_addr + t * C::TILE_BYTES;
+        const uint32_t ka = sKV_addr + kslot * C::TILE_BYTES;
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s) {
+          const uint32_t off = (s >> 2) * C::CHUNK_BYTES + (s & 3) * 32;
+          mma_ss(tmem + t * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), IDESC_S,
+                 s > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, uint32_t vslot, uint32_t acc) {
+        const uint32_t va = sKV_addr + vslot * C::TILE_BYTES;
+#pragma unroll
+        for (int s = 0; s < BN / 16; ++s) {
+          mma_ts(tmem + 256 + t * D, tmem + t * 128 + s * 8, smem_desc_sw128(va + s * 2048, C::CHUNK_BYTES, 1024),
+                 IDESC_O, (s > 0 || acc) ? 1u : 0u);
+        }
+      };
+
+      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_iter) {
+        const Item it = item_at(p, idx);
+        ok = mbar_wait(&q_full, item_iter & 1, w);
+        if (!ok) break;
+        tc_fence_after();
+        const int e = kv_end(p, it);
+        int j = next_union(p, it, 0);
+        bool first_pv[2] = {true, true};
+        if (j < e) {
+          const uint32_t ks = kv_iter % C::NSLOT;
+          ok = mbar_wait(&kv_full[ks], (kv_iter / C::NSLOT) & 1, w);
+          if (!ok) break;
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t) {
+            if (t == 1 && !it.has1) continue;
+            if (!member(p, t == 0 ? it.q0 : it.q1, j)) continue;
+            issue_s(t, ks);
+            tc_commit(&s_full[t]);
+            issued = true;
+          }
+          tc_commit(&kv_empty[ks]);
+          ++kv_iter;
+        }
+        while (ok && j < e) {
+          const int jn = next_union(p, it, j + 1);
+          const uint32_t vs = kv_iter % C::NSLOT;
+          const uint32_t ksn = (kv_iter + 1) % C::NSLOT;
+          ok = mbar_wait(&kv_full[vs], (kv_iter / C::NSLOT) & 1, w);
+          if (ok && jn < e) ok = mbar_wait(&kv_full[ksn], ((kv_iter + 1) / C::NSLOT) & 1, w);
+          if (!ok) break;
+          tc_fence_after();
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (t == 1 && !it.has1) continue;
+            const int qt = t == 0 ? it.q0 : it.q1;
+            if (member(p, qt, j)) {
+              ok = mbar_wait(&p_full[t], p_cnt[t] & 1, w);
+              if (!ok) break;
+              ++p_cnt[t];
+              tc_fence_after();
+              issue_pv(t, vs, first_pv[t] ? 0u : 1u);
+              first_pv[t] = false;
+            }
+            if (jn < e && member(p, qt, jn)) {
+              issue_s(t, ksn);
+              tc_commit(&s_full[t]);
+            }
+          }
+          if (!ok) break;
+          tc_commit(&kv_empty[vs]);
+          if (jn < e) {
+            tc_commit(&kv_empty[ksn]);
+            kv_iter += 2;
+          } else {
+            kv_iter += 1;
+          }
+          j = jn;
+        }
+        if (!ok) break;
+        tc_commit(&o_full[0]);
+        if (it.has1) tc_commit(&o_full[1]);
+        tc_commit(&q_empty);
+      }
+      if (issued) {
+        // Every MMA issued by this thread must be finished before tensor
+        // memory is released.
+        tc_commit(&mma_drain);
+        mbar_drain_wait(&mma_drain, 0, globaltimer_ns() + 100000000ull);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - 4) >> 2;         // query tile of this warpgroup
+    const int quarter = warp & 3;          // tensor-memory lane quarter
+    const int r = quarter * 32 + lane;     // row within the tile
+    const uint32_t lane_bits = uint32_t(quarter * 32) << 16;
+    const uint32_t t_s = tmem + lane_bits + t * 128;
+    const uint32_t t_o = tmem + lane_bits + 256 + t * D;
+    const float sl2 = p.scale_log2;
+    uint32_t s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+
+    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x) {
+      const Item it = item_at(p, idx);
+      if (t == 1 && !it.has1) continue;
+      const int qt = t == 0 ? it.q0 : it.q1;
+      const int row = qt * BM + r;
+      float m = -INFINITY;  // reference maximum, scaled log2 units
+      float l = 0.0f;
+      bool first = true;  // no PV has written this tile's O yet
+      const int e = kv_end(p, it);
+      for (int j = next_union(p, it, 0); j < e; j = next_union(p, it, j + 1)) {
+        if (!member(p, qt, j)) continue;
+        ok = mbar_wait_warp(&s_full[t], s_cnt & 1, w);
+        if (!ok) break;
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t sraw[BN];
+#pragma unroll
+        for (int c = 0; c < BN; c += 32) FA_TMEM_LD_X32(t_s + c, (sraw + c));
+        tc_wait_ld();
+        float x[BN];
+#pragma unroll
+        for (int c = 0; c < BN; ++c) x[c] = __uint_as_float(sraw[c]);
+        const int key0 = j * BN;
+        const bool diag = p.mask_kind == FA_MASK_CAUSAL && j == qt;
+        const int lim = min(diag ? r + 1 : BN, p.N - key0);  // valid columns: [0, lim)
+        if (lim < BN) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c >= lim) x[c] = -INFINITY;
+        }
+        float mx = x[0];
+#pragma unroll
+        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, x[c]);
+        mx *= sl2;
+        const bool grow = mx > m + RESCALE_THRESHOLD;
+        float alpha = 1.0f;
+        if (grow) {
+          alpha = ex2_approx(m - mx);  // 0 when m == -inf
+          m = mx;
+          l *= alpha;
+        }
+        if (__any_sync(0xffffffffu, grow && !first)) {
+          // The reference maximum moved for some row of this warp: bring its
+          // O accumulator onto the new reference (rows that did not move
+          // multiply by 1).  Before the first PV of an item there is nothing
+          // to rescale: that PV overwrites O.
+          const float a = (grow && !first) ? alpha : 1.0f;
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t v[32];
+            FA_TMEM_LD_X32(t_o + c, v);
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
+            FA_TMEM_ST_X32(t_o + c, v);
+          }
+        }
+        first = false;
+        const float m_use = (m == -INFINITY) ? 0.0f : m;
+        float rs = 0.0f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = ex2_approx(fmaf(x[64 * h + 2 * i], sl2, -m_use));
+            const float p1 = ex2_approx(fmaf(x[64 * h + 2 * i + 1], sl2, -m_use));
+            rs += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          FA_TMEM_ST_X32(t_s + 32 * h, pk);
+        }
+        l += rs;
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l and LSE
+      ok = mbar_wait_warp(&o_full[t], o_cnt & 1, w);
+      if (!ok) break;
+      ++o_cnt;
+      tc_fence_after();
+      const bool live = l > 0.0f;  // false only for a row that sees no key
+      const float inv_l = live ? 1.0f / l : 0.0f;
+      __nv_bfloat16* orow = p.O + ((size_t)it.bh * p.N + row) * D;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t v[32];
+        FA_TMEM_LD_X32(t_o + c, v);
+        tc_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = live ? pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l) : 0u;
+        if (row < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      if (row < p.N) p.LSE[(size_t)it.bh * p.N + row] = live ? (m + log2f(l)) * LN2 : -INFINITY;
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fwd
+
+fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void* V, void* O, float* LSE,
+                     cudaStream_t s) {
+  uint32_t* st = status_word();
+  if (!st) return FA_ERR_CUDA;
+  CUtensorMap mQ, mK, mV;
+  if (!make_map_bf16(&mQ, Q, pr.BH, pr.N, pr.d, fwd::BM) || !make_map_bf16(&mK, K, pr.BH, pr.N, pr.d, fwd::BN) ||
+      !make_map_bf16(&mV, V, pr.BH, pr.N, pr.d, fwd::BN))
+    return FA_ERR_CUDA;
+  fwd::Params p;
+  p.BH = pr.BH;
+  p.N = pr.N;
+  p.nq = pr.nq;
+  p.n_pairs = (pr.nq + 1) / 2;
+  p.n_items = p.n_pairs * pr.BH;
+  p.mask_kind = pr.mask_kind;
+  p.block_mask = pr.block_mask;
+  p.scale_log2 = pr.scale_log2;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.LSE = LSE;
+  p.timeout_ns = wait_timeout_ns();
+  p.status = st;
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  if (pr.d == 64) {
+    constexpr int smem = fwd::Cfg<64>::SMEM_BYTES;
+    if (cudaFuncSetAttribute(fwd::fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return FA_ERR_CUDA;
+    fwd::fwd_kernel<64><<<grid, fwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, p);
+  } else {
+    constexpr int smem = fwd::Cfg<128>::SMEM_BYTES;
+    if (cudaFuncSetAttribute(fwd::fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return FA_ERR_CUDA;
+    fwd::fwd_kernel<128><<<grid, fwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, p);
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace fa

@@ -1,0 +1,128 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact, IO-aware scaled-dot-product attention
+ * (forward and backward) for NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  For every head (b, h) of [B, H, N, d] tensors:
+ *     S = scale * Q K^T   (with a mask applied as -inf),
+ *     P = softmax(S) row by row,   O = P V,   LSE_i = ln sum_j exp(S_ij).
+ * The method is the one described on the pages "FlashAttention: making
+ * attention fast by respecting the memory hierarchy" (tiling paragraph:
+ * blocks of queries against blocks of keys and values, an online softmax,
+ * the full score grid never written to slow memory) and "FlashAttention:
+ * Fast and Memory-Efficient Exact Attention with IO-Awareness" (sections
+ * "What FlashAttention targets": exact, same outputs as naive attention;
+ * "Softmax / tiling"; "Backward / recomputation": the forward stores the
+ * softmax normalisation statistics -- here the per-row log-sum-exp -- and the
+ * backward recomputes the attention values on chip from them).
+ *
+ * Conventions shared by every call:
+ *   - Q, K, V, O, dO, dQ, dK, dV: bf16, contiguous [B, H, N, d] (d fastest),
+ *     DEVICE pointers, 16-byte aligned.  N_q = N_k = N (self-attention).
+ *   - LSE: fp32 [B, H, N], natural log, DEVICE pointer, 4-byte aligned.
+ *   - d must be 64 or 128.  N >= 1 is any length (a last partial tile of
+ *     128 rows is handled by masking).
+ *   - mask_kind: FA_MASK_NONE, FA_MASK_CAUSAL (key j visible to query i iff
+ *     j <= i, top-left aligned) or FA_MASK_BLOCK.  For FA_MASK_BLOCK,
+ *     `block_mask` is a DEVICE uint8 array [nb, nb], nb = ceil(N / 128),
+ *     row-major, entry (I, J) != 0 keeping the 128 x 128 score tile of query
+ *     rows [128 I, 128 I + 128) and key columns [128 J, 128 J + 128); one mask
+ *     serves every batch and head (block-sparse FlashAttention, "Paper
+ *     Abstract" of the summary page).  It is ignored for the other kinds.
+ *     A query row with no visible key gets O = 0, LSE = -inf, and contributes
+ *     nothing to the gradients.
+ *   - scale: finite, > 0 (usually 1/sqrt(d)).
+ *   - stream: a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Every call is asynchronous on it.
+ *   - Ownership: the caller allocates and owns every buffer and the stream;
+ *     the library keeps no allocation between calls.
+ *   - Outputs must not alias inputs.
+ *   - Errors: argument problems are reported synchronously, before anything
+ *     is launched.  A failed launch returns FA_ERR_CUDA.  Every wait inside
+ *     the kernels is bounded in time; a wait that runs out records
+ *     FA_ERR_TIMEOUT in a per-device status word that fa_device_status()
+ *     reads (the outputs of that call are then undefined).
+ */
+#ifndef FA_H
+#define FA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, bad scale, bad mask kind */
+  FA_ERR_UNSUPPORTED = 2, /* valid request outside this build: d not 64/128, sizes beyond int range */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed */
+  FA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than fa_bwd_workspace_size() */
+  FA_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out (see fa_device_status) */
+} fa_status;
+
+typedef enum { FA_MASK_NONE = 0, FA_MASK_CAUSAL = 1, FA_MASK_BLOCK = 2 } fa_mask_kind;
+
+/* Forward pass.
+ * In:  Q, K, V [B,H,N,d] bf16; mask (kind + optional device block mask); scale.
+ * Out: O [B,H,N,d] bf16 (round to nearest even); LSE [B,H,N] fp32, the
+ *      natural-log normaliser of the scaled, masked scores of each row.
+ * The N x N score grid never leaves the chip. */
+fa_status fa_fwd(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                 int mask_kind, const uint8_t* block_mask, float scale, void* O, float* LSE,
+                 void* stream);
+
+/* Bytes of device workspace fa_bwd needs for this problem size: an fp32 dQ
+ * accumulator [B,H,ceil(N/128)*128,d], the fp32 row terms D_i = dO_i . O_i
+ * [B,H,ceil(N/128)*128], plus alignment padding.  Linear in N.  Returns 0 for
+ * sizes fa_bwd would reject. */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/* Backward pass, recomputing P on chip from Q, K and the forward's LSE.
+ * In:  Q, K, V, O, dO [B,H,N,d] bf16; LSE [B,H,N] fp32 from fa_fwd with the
+ *      same mask and scale; workspace (DEVICE, 256-byte aligned, at least
+ *      fa_bwd_workspace_size() bytes, contents irrelevant on entry).
+ * Out: dQ, dK, dV [B,H,N,d] bf16, gradients of sum(dO * O) with respect to
+ *      Q, K and V.  dQ is summed over key tiles in fp32 in an unspecified
+ *      order, so its last bits may differ from run to run. */
+fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                 const float* LSE, int B, int H, int N, int d, int mask_kind,
+                 const uint8_t* block_mask, float scale, void* dQ, void* dK, void* dV,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, then read and clear the calling device's status
+ * word.  Returns FA_OK, FA_ERR_TIMEOUT if a bounded wait ran out in a kernel
+ * since the last call, or FA_ERR_CUDA if the synchronisation itself failed. */
+fa_status fa_device_status(void* stream);
+
+/* Set the wall-clock limit, in nanoseconds, of every device-side wait in
+ * later launches from this process (default 4e9 = 4 s).  0 restores the
+ * default. */
+void fa_set_wait_timeout_ns(uint64_t ns);
+
+/* Human-readable name of a status code (static string). */
+const char* fa_status_string(fa_status s);
+
+/* Self-test of the bounded-wait machinery: launches one CTA whose thread
+ * waits, for at most `timeout_ns`, on an mbarrier that nothing ever
+ * completes, then returns.  After fa_device_status() the caller should see
+ * FA_ERR_TIMEOUT.  No page counterpart: this exercises the library's own
+ * failure detection. */
+fa_status fa_selftest_bounded_wait(uint64_t timeout_ns, void* stream);
+
+/* Self-test of the tensor-core path on one tile, used to validate the
+ * shared-memory/TMEM descriptors in isolation.  A [128 x k] and Bt
+ * [n x k] are bf16 row-major DEVICE arrays (k in {64, 128}; n in {64, 128});
+ * C [128 x n] fp32 DEVICE receives A * Bt^T computed by TMA loads plus one
+ * tcgen05.mma chain from shared memory (mode 0), or, in mode 1, by first
+ * packing A into tensor memory and multiplying by Bt read as an MN-major
+ * [k x n] operand -- the two forms that S = Q K^T and O += P V take. In
+ * mode 1, B is passed as [k x n] row-major instead.  No page counterpart. */
+fa_status fa_selftest_mma_tile(const void* A, const void* B, float* C, int n, int k, int mode,
+                               void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H */

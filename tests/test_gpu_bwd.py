@@ -1,0 +1,104 @@
+"""Backward parity: fa_bwd through the C ABI against the fp64 oracle's
+gradients on the same seeded bf16 inputs."""
+import numpy as np
+import pytest
+import torch
+
+import exact_io_aware_65_b200 as fa
+import oracle
+import workloads
+from helpers import has_gpu, to_dev, f64, assert_grad, GRAD_REL_L2
+
+pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not has_gpu(), reason="needs a B200")]
+
+SMALL = [
+    (1, 1, 128, 64, "none"),
+    (1, 1, 1, 64, "none"),
+    (1, 1, 1, 128, "causal"),
+    (2, 3, 300, 64, "none"),
+    (2, 3, 300, 64, "causal"),
+    (2, 3, 300, 64, "block"),
+    (1, 2, 640, 128, "causal"),
+    (1, 2, 257, 128, "none"),
+    (1, 2, 383, 128, "block"),
+    (3, 1, 127, 64, "causal"),
+    (1, 1, 129, 128, "causal"),
+    (2, 2, 1024, 64, "causal"),
+    (1, 2, 1024, 128, "none"),
+]
+
+
+def run(w, x, O=None, L=None):
+    d = to_dev(x)
+    if O is None:
+        O, L = fa.fwd(d["Q"], d["K"], d["V"], w.mask, d["mask"], w.scale)
+    g = fa.bwd(d["Q"], d["K"], d["V"], O, d["dO"], L, w.mask, d["mask"], w.scale)
+    assert fa.device_status() == 0
+    return g
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=[f"{b}x{h}x{n}x{d}-{m}" for b, h, n, d, m in SMALL])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_bwd_small(shape, seed):
+    B, H, N, d, m = shape
+    w = workloads.Workload("t", B, H, N, d, m, float(np.float32(d ** -0.5)))
+    x = workloads.make_inputs(w, seed)
+    dQ, dK, dV = run(w, x)
+    ref = oracle.bwd(x["Q"], x["K"], x["V"], x["dO"], m, x["mask"], w.scale)
+    for name, g in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        assert_grad(f64(g), ref[name], name, str(shape))
+
+
+@pytest.mark.parametrize("shape", [(2, 3, 300, 64, "causal"), (1, 2, 383, 128, "block")])
+def test_bwd_from_oracle_statistics(shape):
+    """Feed the oracle's O (rounded to bf16) and LSE (fp32) to isolate the
+    backward's own error from the forward's."""
+    B, H, N, d, m = shape
+    w = workloads.Workload("t", B, H, N, d, m, float(np.float32(d ** -0.5)))
+    x = workloads.make_inputs(w, 5)
+    ref = oracle.bwd(x["Q"], x["K"], x["V"], x["dO"], m, x["mask"], w.scale)
+    O = torch.from_numpy(ref["O"]).to(torch.bfloat16).cuda()
+    L = torch.from_numpy(ref["LSE"]).to(torch.float32).cuda()
+    dQ, dK, dV = run(w, x, O, L)
+    for name, g in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        assert_grad(f64(g), ref[name], name, str(shape))
+
+
+def test_bwd_block_mask_with_empty_rows_and_columns():
+    w = workloads.Workload("t", 1, 2, 384, 64, "block", 0.125)
+    x = workloads.make_inputs(w, 6)
+    x["mask"] = torch.tensor([[1, 0, 1], [0, 0, 0], [0, 0, 1]], dtype=torch.uint8)
+    dQ, dK, dV = run(w, x)
+    ref = oracle.bwd(x["Q"], x["K"], x["V"], x["dO"], "block", x["mask"], w.scale)
+    assert (f64(dQ)[:, :, 128:256] == 0).all()      # query block that sees nothing
+    assert (f64(dK)[:, :, 128:256] == 0).all()      # key block nobody sees
+    assert (f64(dV)[:, :, 128:256] == 0).all()
+    for name, g in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        assert_grad(f64(g), ref[name], name)
+
+
+@pytest.mark.parametrize("mask", ["none", "causal", "block"])
+def test_bwd_gradient_identities(mask):
+    """Properties that hold at any size: rows of dS sum to zero, so sum_j dK_j
+    = 0; rows of P sum to one, so sum_j dV_j = sum_i dO_i."""
+    w = workloads.Workload("t", 2, 2, 1024, 128, mask, float(np.float32(128 ** -0.5)))
+    x = workloads.make_inputs(w, 7)
+    dQ, dK, dV = run(w, x)
+    dk, dv, do = f64(dK), f64(dV), f64(x["dO"])
+    scale_k = np.abs(dk).sum(axis=2).max()
+    assert np.abs(dk.sum(axis=2)).max() <= 2e-2 * scale_k
+    np.testing.assert_allclose(dv.sum(axis=2), do.sum(axis=2), atol=2e-2 * np.abs(do).sum(axis=2).max())
+
+
+@pytest.mark.parametrize("name", workloads.ORDER)
+def test_bwd_workloads_one_head(name):
+    """Full-size workloads in the benchmark's launch configuration; the
+    oracle recomputes one whole head (heads are independent)."""
+    w = workloads.WORKLOADS[name]
+    x = workloads.make_inputs(w, 0)
+    dQ, dK, dV = run(w, x)
+    h = w.B * w.H - 1
+    sl = lambda t: t.reshape(w.B * w.H, w.N, w.d)[h:h + 1]
+    ref = oracle.bwd(sl(x["Q"]), sl(x["K"]), sl(x["V"]), sl(x["dO"]), w.mask, x["mask"], w.scale)
+    for nm, g in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        assert_grad(f64(sl(g)), ref[nm][0:1], nm, name)
