@@ -33,6 +33,8 @@ SIGNATURES = {
     "fa_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp]),
     "fa_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
     "fa_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "fa_bwd_stage": (_i, [_i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp, _vp,
+                          _sz, _vp]),
     "fa_device_status": (_i, [_vp]),
     "fa_set_wait_timeout_ns": (None, [_u64]),
     "fa_status_string": (ctypes.c_char_p, [_i]),
@@ -130,6 +132,19 @@ def bwd(Q, K, V, O, dO, LSE, mask="none", block_mask=None, scale=None, dQ=None, 
                         dV.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)),
            "fa_bwd")
     return dQ, dK, dV
+
+
+def bwd_stage(stage, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, mask="none", block_mask=None,
+              scale=None, stream=None):
+    """One of the three launches of ``bwd`` (0: prep, 1: main, 2: dQ
+    convert); running 0, 1, 2 in order on one workspace equals ``bwd``."""
+    B, H, N, d = Q.shape
+    scale = d ** -0.5 if scale is None else float(scale)
+    kind, mptr = _mask(mask, block_mask)
+    _check(lib().fa_bwd_stage(int(stage), Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(),
+                              dO.data_ptr(), LSE.data_ptr(), B, H, N, d, kind, mptr, scale, dQ.data_ptr(),
+                              dK.data_ptr(), dV.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                              _stream(stream)), f"fa_bwd_stage({stage})")
 
 
 def device_status(stream=None) -> int:

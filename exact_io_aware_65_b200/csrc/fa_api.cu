@@ -119,9 +119,10 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return bwd_workspace_bytes(B, H, N, d);
 }
 
-fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
-                 int B, int H, int N, int d, int mask_kind, const uint8_t* block_mask, float scale, void* dQ,
-                 void* dK, void* dV, void* workspace, size_t workspace_bytes, void* stream) {
+static fa_status bwd_common(int stage, const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                            const float* LSE, int B, int H, int N, int d, int mask_kind, const uint8_t* block_mask,
+                            float scale, void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes,
+                            void* stream) {
   Problem p;
   fa_status st = check_common(Q, K, V, B, H, N, d, mask_kind, block_mask, scale, &p);
   if (st != FA_OK) return st;
@@ -131,7 +132,23 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
     return FA_ERR_INVALID_ARG;
   const size_t need = bwd_workspace_bytes(B, H, N, d);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FA_ERR_WORKSPACE;
-  return launch_bwd(p, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, (cudaStream_t)stream);
+  return launch_bwd(p, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, (cudaStream_t)stream, stage);
+}
+
+fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                 int B, int H, int N, int d, int mask_kind, const uint8_t* block_mask, float scale, void* dQ,
+                 void* dK, void* dV, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_common(-1, Q, K, V, O, dO, LSE, B, H, N, d, mask_kind, block_mask, scale, dQ, dK, dV, workspace,
+                    workspace_bytes, stream);
+}
+
+fa_status fa_bwd_stage(int stage, const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                       const float* LSE, int B, int H, int N, int d, int mask_kind, const uint8_t* block_mask,
+                       float scale, void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  if (stage < 0 || stage > 2) return FA_ERR_INVALID_ARG;
+  return bwd_common(stage, Q, K, V, O, dO, LSE, B, H, N, d, mask_kind, block_mask, scale, dQ, dK, dV, workspace,
+                    workspace_bytes, stream);
 }
 
 fa_status fa_device_status(void* stream) {

@@ -208,6 +208,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   __shared__ __align__(8) uint64_t kv_full, kv_empty, s_full, p_full, ds_full, dkdv_full, mma_drain;
+  // The two column halves of a lane quarter write their packed bf16 results
+  // into columns the other half may still be reading as fp32: each half
+  // arrives once its loads are done and waits for the other before storing.
+  __shared__ __align__(8) uint64_t s_read, dp_read;
   __shared__ __align__(8) uint64_t qd_full[C::NST], qd_empty[C::NST], dq_full[C::NDQ], dq_free[C::NDQ];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -222,6 +226,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(&ds_full, 256);
     mbar_init(&dkdv_full, 1);
     mbar_init(&mma_drain, 1);
+    mbar_init(&s_read, 256);
+    mbar_init(&dp_read, 256);
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(&qd_full[s], 1);
       mbar_init(&qd_empty[s], 1);
@@ -396,20 +402,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool key_live = key < p.N;
         const bool diag = p.mask_kind == FA_MASK_CAUSAL && i == it.j;
         float pr[64];
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t sr[32];
-          FA_TMEM_LD_X32(tmem + lane_bits + C::COL_S + hf * 64 + cc * 32, sr);
+        {
+          uint32_t sr[64];
+          FA_TMEM_LD_X32(tmem + lane_bits + C::COL_S + hf * 64, sr);
+          FA_TMEM_LD_X32(tmem + lane_bits + C::COL_S + hf * 64 + 32, (sr + 32));
           tc_wait_ld();
-          const float4* l4 = reinterpret_cast<const float4*>(p.L2w + rowbase + cc * 32);
+          tc_fence_before();
+          mbar_arrive(&s_read);
+          const float4* l4 = reinterpret_cast<const float4*>(p.L2w + rowbase);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
+          for (int u = 0; u < 16; ++u) {
             const float4 lv = __ldg(l4 + u);
             const float lvv[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int col = cc * 32 + u * 4 + e;
-              float pv = ex2_approx(fmaf(__uint_as_float(sr[u * 4 + e]), sl2, -lvv[e]));
+              const int col = u * 4 + e;
+              float pv = ex2_approx(fmaf(__uint_as_float(sr[col]), sl2, -lvv[e]));
               if (!key_live || (diag && hf * 64 + col < kr)) pv = 0.0f;
               pr[col] = pv;
             }
@@ -419,6 +427,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
+          ok = mbar_wait_warp(&s_read, (s_cnt - 1) & 1, w);
+          if (!ok) break;
+          tc_fence_after();
           FA_TMEM_ST_X32(tmem + lane_bits + C::COL_S + hf * 32, pk);
         }
         tc_wait_st();
@@ -426,13 +437,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive(&p_full);
         // dS^T = P^T * (dP^T - D)
         uint8_t* ds_chunk = sDS + hf * C::CHUNK_BYTES + kr * 128;
+        uint32_t dk[32];
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           uint32_t dr[32];
           FA_TMEM_LD_X32(tmem + lane_bits + C::COL_DP + hf * 64 + cc * 32, dr);
           tc_wait_ld();
+          if (cc == 1) {
+            tc_fence_before();
+            mbar_arrive(&dp_read);
+          }
           const float4* d4 = reinterpret_cast<const float4*>(p.Dw + rowbase + cc * 32);
-          uint32_t pk[16];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const float4 dv = __ldg(d4 + u);
@@ -441,19 +456,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float g1 = pr[c + 1] * (__uint_as_float(dr[u * 4 + 1]) - dv.y);
             const float g2 = pr[c + 2] * (__uint_as_float(dr[u * 4 + 2]) - dv.z);
             const float g3 = pr[c + 3] * (__uint_as_float(dr[u * 4 + 3]) - dv.w);
-            pk[u * 2 + 0] = pack_bf16x2(g0, g1);
-            pk[u * 2 + 1] = pack_bf16x2(g2, g3);
-          }
-          FA_TMEM_ST_X16(tmem + lane_bits + C::COL_DP + hf * 32 + cc * 16, pk);
-          // shared-memory copy, 128-byte swizzle: 16-byte unit u of row kr
-          // lives at unit (u ^ (kr & 7)).
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int unit = (cc * 4 + u) ^ (kr & 7);
-            *reinterpret_cast<uint4*>(ds_chunk + unit * 16) =
-                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+            dk[cc * 16 + u * 2 + 0] = pack_bf16x2(g0, g1);
+            dk[cc * 16 + u * 2 + 1] = pack_bf16x2(g2, g3);
           }
         }
+        // shared-memory copy of dS^T, 128-byte swizzle: 16-byte unit u of
+        // row kr lives at unit (u ^ (kr & 7)).
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int unit = u ^ (kr & 7);
+          *reinterpret_cast<uint4*>(ds_chunk + unit * 16) =
+              make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+        }
+        ok = mbar_wait_warp(&dp_read, (s_cnt - 1) & 1, w);
+        if (!ok) break;
+        tc_fence_after();
+        FA_TMEM_ST_X32(tmem + lane_bits + C::COL_DP + hf * 32, dk);
         tc_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
@@ -547,7 +565,7 @@ size_t bwd_workspace_bytes(int B, int H, int N, int d) {
 template <int D>
 static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CUtensorMap& mK, const CUtensorMap& mV,
                               const CUtensorMap& mdO, const void* O, const void* dO, const float* LSE, void* dQ,
-                              void* dK, void* dV, void* workspace, cudaStream_t s, uint32_t* st) {
+                              void* dK, void* dV, void* workspace, cudaStream_t s, uint32_t* st, int stage) {
   const int Npad = pr.nq * 128;
   const bwd::Workspace wl = bwd::workspace_layout(pr.BH, Npad, D);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -556,7 +574,7 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
   float* L2w = reinterpret_cast<float*>(ws + wl.l2_off);
   const int sms = num_sms();
 
-  {
+  if (stage < 0 || stage == 0) {
     const long long rows = (long long)pr.BH * Npad;
     const long long warps_needed = (rows + (32 / (D / 8)) - 1) / (32 / (D / 8));
     long long blocks = (warps_needed + 7) / 8;
@@ -566,7 +584,7 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
                                                      pr.BH, pr.N, Npad);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
-  {
+  if (stage < 0 || stage == 1) {
     bwd::Params p;
     p.BH = pr.BH;
     p.N = pr.N;
@@ -591,7 +609,7 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     bwd::main_kernel<D><<<grid, bwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, mdO, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
-  {
+  if (stage < 0 || stage == 2) {
     const long long work = (long long)pr.BH * pr.N * (D / 8);
     long long blocks = (work + 255) / 256;
     if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
@@ -603,15 +621,15 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
 }
 
 fa_status launch_bwd(const Problem& pr, const void* Q, const void* K, const void* V, const void* O, const void* dO,
-                     const float* LSE, void* dQ, void* dK, void* dV, void* workspace, cudaStream_t s) {
+                     const float* LSE, void* dQ, void* dK, void* dV, void* workspace, cudaStream_t s, int stage) {
   uint32_t* st = status_word();
   if (!st) return FA_ERR_CUDA;
   CUtensorMap mQ, mK, mV, mdO;
   if (!make_map_bf16(&mQ, Q, pr.BH, pr.N, pr.d, 128) || !make_map_bf16(&mK, K, pr.BH, pr.N, pr.d, 128) ||
       !make_map_bf16(&mV, V, pr.BH, pr.N, pr.d, 128) || !make_map_bf16(&mdO, dO, pr.BH, pr.N, pr.d, 128))
     return FA_ERR_CUDA;
-  if (pr.d == 64) return launch_bwd_d<64>(pr, mQ, mK, mV, mdO, O, dO, LSE, dQ, dK, dV, workspace, s, st);
-  return launch_bwd_d<128>(pr, mQ, mK, mV, mdO, O, dO, LSE, dQ, dK, dV, workspace, s, st);
+  if (pr.d == 64) return launch_bwd_d<64>(pr, mQ, mK, mV, mdO, O, dO, LSE, dQ, dK, dV, workspace, s, st, stage);
+  return launch_bwd_d<128>(pr, mQ, mK, mV, mdO, O, dO, LSE, dQ, dK, dV, workspace, s, st, stage);
 }
 
 }  // namespace fa

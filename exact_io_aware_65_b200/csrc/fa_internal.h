@@ -36,9 +36,10 @@ int num_sms();
 // Kernel launchers (defined next to their kernels).
 fa_status launch_fwd(const Problem& p, const void* Q, const void* K, const void* V, void* O, float* LSE,
                      cudaStream_t s);
+// stage < 0: all three stages; otherwise only the given one (0, 1 or 2).
 fa_status launch_bwd(const Problem& p, const void* Q, const void* K, const void* V, const void* O,
                      const void* dO, const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
-                     cudaStream_t s);
+                     cudaStream_t s, int stage);
 size_t bwd_workspace_bytes(int B, int H, int N, int d);
 fa_status launch_selftest_wait(uint64_t timeout_ns, cudaStream_t s);
 fa_status launch_selftest_mma(const void* A, const void* B, float* C, int n, int k, int mode, cudaStream_t s);
