@@ -1,0 +1,363 @@
+#!/usr/bin/env python
+"""Benchmark exact attention (forward and forward+backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: fa_fwd, then the
+three launches of fa_bwd (prep, main, dQ convert).  The default workload is
+the long causal context (B=2, H=16, N=8192, d=128), the one the forward +
+backward throughput target is stated for.  `value` is algorithmic TFLOP/s of
+forward + backward summed over all ranks (4 d flops per kept score entry
+forward, 10 d backward); with N > 1 every rank runs its own replica of the
+workload (heads are independent, so there is no data-path collective) and
+the time is the maximum over ranks.
+
+`--impl reference` times the fp64 CPU oracle on this host instead (rank 0
+only), on a bounded sample of the same workload per step.
+
+Prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "attention fwd and fwd+bwd TFLOP/s (bf16) and % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "long_s8k_d128_causal"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def flops(w: workloads.Workload, mask) -> dict:
+    E = workloads.kept_entries(w, mask)
+    per = w.B * w.H * E * w.d
+    return {"fwd": 4 * per, "bwd": 10 * per, "E": E}
+
+
+def source_sha(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current source of that kernel (else None)."""
+    f = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(f):
+        return None
+    rec = json.load(open(f)).get(kernel, {}).get(workload)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src) or source_sha(src) != rec["source_sha"]:
+        return None
+    return rec["dram_bytes_per_launch"]
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons (read only)."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.t0 = self.t1 = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={ident}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(1.0)
+        except Exception:
+            self.proc = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def result(self):
+        if self.proc is None:
+            return {"error": "nvidia-smi unavailable"}
+        time.sleep(0.3)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[4:8]))
+            except ValueError:
+                continue
+        inside = [r for r in rows if self.t0 - 1 <= r[0] <= self.t1 + 1] or rows
+        if not inside:
+            return {"error": "no samples"}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in inside for n, v in zip(names, r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside)}
+
+
+def cpu_sample(w, x, mask, seed_rows=None):
+    """Time the fp64 oracle (fwd + bwd) on one head of the workload,
+    truncated to its first `n` positions; returns (TFLOP/s, seconds, desc)."""
+    import oracle  # test infrastructure: only the CPU-baseline leg uses it
+
+    n = seed_rows or w.N
+    sl = lambda t: t.reshape(w.B * w.H, w.N, w.d)[:1, :n].contiguous()
+    sub = w.with_(B=1, H=1, N=n)
+    m = mask[: sub.nb, : sub.nb].contiguous() if mask is not None else None
+    t0 = time.perf_counter()
+    oracle.bwd(sl(x["Q"]), sl(x["K"]), sl(x["V"]), sl(x["dO"]), w.mask, m, w.scale)
+    dt = time.perf_counter() - t0
+    f = flops(sub, m)
+    desc = (f"fp64 oracle fwd+bwd (plain definition, all masked entries skipped) on head 0 of "
+            f"{w.name}, first {n} of {w.N} positions ({f['E']} kept score entries)")
+    return (f["fwd"] + f["bwd"]) / dt / 1e12, dt, desc, oracle.num_threads()
+
+
+def reference_arm(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    x = workloads.make_inputs(w, args.seed)
+    n = min(w.N, 2048)
+    for _ in range(args.warmup):
+        cpu_sample(w, x, x["mask"], n)
+    vals, secs = [], 0.0
+    desc = cores = None
+    for _ in range(args.steps):
+        v, dt, desc, cores = cpu_sample(w, x, x["mask"], n)
+        vals.append(v)
+        secs += dt
+    value = (args.steps * (flops(w.with_(B=1, H=1, N=n), x["mask"])["fwd"] +
+                           flops(w.with_(B=1, H=1, N=n), x["mask"])["bwd"])) / secs / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": desc + " per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "mask": w.mask, "scale": w.scale}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=workloads.ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = workloads.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return reference_arm(args, w)
+
+    import exact_io_aware_65_b200 as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if dist is None:
+            return v
+        t = torch.tensor([v], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- inputs resident in HBM (each rank its own replica of the workload)
+    x = workloads.make_inputs(w, args.seed + rank)
+    mask_cpu = x["mask"]
+    Q, K, V, dO = (x[n].to(dev) for n in ("Q", "K", "V", "dO"))
+    mask = mask_cpu.to(dev) if mask_cpu is not None else None
+    O = torch.empty_like(Q)
+    LSE = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    ws = torch.empty(fa.bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    names = ("fwd", "bwd_prep", "bwd_main", "bwd_dq_convert")
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        fa.fwd(Q, K, V, w.mask, mask, w.scale, O=O, LSE=LSE, stream=stream)
+        if evs is not None:
+            evs[1].record(stream)
+        for s in range(3):
+            fa.bwd_stage(s, Q, K, V, O, dO, LSE, dQ, dK, dV, ws, w.mask, mask, w.scale, stream=stream)
+            if evs is not None:
+                evs[2 + s].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if fa.device_status() != 0:
+        raise SystemExit("device status reports a timed-out wait during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.mark_start()
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks.mark_end()
+    status = fa.device_status()
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    per_kernel = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(names)}
+    clock_info = clocks.result()
+
+    fl = flops(w, mask_cpu)
+    ms_step = total_ms / args.steps
+    value = world * (fl["fwd"] + fl["bwd"]) / (ms_step * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    fwd_tflops = fl["fwd"] / (per_kernel["fwd"] * 1e-3) / 1e12
+    bwd_ms = per_kernel["bwd_prep"] + per_kernel["bwd_main"] + per_kernel["bwd_dq_convert"]
+    bwd_tflops = fl["bwd"] / (bwd_ms * 1e-3) / 1e12
+
+    # dominant kernel and its roofline (tensor-bound contraction)
+    dom = max(("fwd", "bwd_main"), key=lambda n: per_kernel[n])
+    dom_flops = fl["fwd"] if dom == "fwd" else fl["bwd"]
+    achieved = dom_flops / (per_kernel[dom] * 1e-3) / 1e12
+    dom_src = {"fwd": "exact_io_aware_65_b200/csrc/fa_fwd.cu", "bwd_main": "exact_io_aware_65_b200/csrc/fa_bwd.cu"}
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                "peak_source": f"{peak_kind} bf16 dense (burst)",
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                "traffic": traffic_for(dom, w.name), "source": dom_src[dom]}
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = args.e2e_steps or max(3, min(args.steps, 30))
+    hostin = {n: x[n].pin_memory() for n in ("Q", "K", "V", "dO")}
+    host_mask = mask_cpu.pin_memory() if mask_cpu is not None else None
+    hostout = {"O": torch.empty_like(O, device="cpu").pin_memory(),
+               "LSE": torch.empty_like(LSE, device="cpu").pin_memory(),
+               "dQ": torch.empty_like(dQ, device="cpu").pin_memory(),
+               "dK": torch.empty_like(dK, device="cpu").pin_memory(),
+               "dV": torch.empty_like(dV, device="cpu").pin_memory()}
+    dev_in = {n: torch.empty_like(hostin[n], device=dev) for n in hostin}
+    dev_mask = torch.empty_like(host_mask, device=dev) if host_mask is not None else None
+    h2d = sum(t.numel() * t.element_size() for t in hostin.values()) + (host_mask.numel() if host_mask is not None else 0)
+    d2h = sum(t.numel() * t.element_size() for t in hostout.values())
+
+    def e2e_step():
+        for n in hostin:
+            dev_in[n].copy_(hostin[n], non_blocking=True)
+        if dev_mask is not None:
+            dev_mask.copy_(host_mask, non_blocking=True)
+        o, lse = fa.fwd(dev_in["Q"], dev_in["K"], dev_in["V"], w.mask, dev_mask, w.scale, O=O, LSE=LSE,
+                        stream=stream)
+        fa.bwd(dev_in["Q"], dev_in["K"], dev_in["V"], o, dev_in["dO"], lse, w.mask, dev_mask, w.scale,
+               dQ=dQ, dK=dK, dV=dV, workspace=ws, stream=stream)
+        for n, src in (("O", O), ("LSE", LSE), ("dQ", dQ), ("dK", dK), ("dV", dV)):
+            hostout[n].copy_(src, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+    e2e_value = world * (fl["fwd"] + fl["bwd"]) / (e2e_ms * 1e-3) / 1e12
+    status = status or fa.device_status()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, dt, desc, cores = cpu_sample(w, x, mask_cpu)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc, "seconds": dt}
+
+    in_bytes = sum(t.numel() * t.element_size() for t in (Q, K, V, dO, O, LSE, dQ, dK, dV)) + ws.numel()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded i.i.d. N(0,1) Q, K, V, dO rounded to bf16 (no dataset)",
+        "config": dict(workload_config(w), parallelism=f"{world} independent replica(s), one per GPU",
+                       l2=f"no flush: step touches {in_bytes / 2**20:.0f} MiB, more than the "
+                          f"{L2_BYTES / 2**20:.0f} MiB L2"),
+        "fwd": {"ms": per_kernel["fwd"], "tflops": fwd_tflops, "frac_of_peak": fwd_tflops / peaks["bf16_tflops"]},
+        "fwd_bwd": {"ms": ms_step, "tflops": value / world, "frac_of_peak": value / world / peaks["bf16_tflops"]},
+        "bwd": {"ms": bwd_ms, "tflops": bwd_tflops},
+        "kernels_ms": per_kernel,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms, "steps": e2e_steps},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clock_info,
+        "device_status": status,
+        "peaks": {"bf16_tflops": peaks["bf16_tflops"], "bf16_tflops_sustained": peaks["bf16_tflops_sustained"],
+                  "source": peak_kind},
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    if status != 0:
+        raise SystemExit(f"device status {status}: a bounded wait timed out")
+
+
+if __name__ == "__main__":
+    main()

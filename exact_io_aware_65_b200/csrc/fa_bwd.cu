@@ -30,10 +30,11 @@
 // CTA roles (512 threads): warp 0 TMA producer; warp 1 MMA issuer; warps
 // 4..11 softmax (thread = key row; warps 4..7 take query columns 0..63,
 // warps 8..11 columns 64..127); warps 12..15 dQ drain (thread = query row).
-// Tensor memory: S^T [0,128) then P^T (bf16) in [0,64); dP^T [128,256) then
-// dS^T (bf16) in [128,192); dV [256, 256+d); dK [256+d, 256+2d).  The dQ
-// tile sits in the columns P and dS left free ([64,128) and [192,256)) for
-// d = 128, and in two buffers at [384,448) and [448,512) for d = 64.
+// Tensor memory: S^T [0,128), then P^T (bf16) in [0,64) and dS^T (bf16) in
+// [64,128); dP^T [128,256); dV [256, 256+d); dK [256+d, 256+2d).  The dQ
+// tile reuses the dP^T columns for d = 128 (so the next dP^T waits for the
+// drain, the next S^T does not), and has two buffers at [384,448) and
+// [448,512) for d = 64.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -50,16 +51,21 @@ constexpr float LOG2E = 1.4426950408889634074f;
 
 __host__ __device__ constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Workspace carve-up (all offsets 256-byte aligned).
+// Workspace carve-up (all offsets 256-byte aligned).  The fp32 dQ
+// accumulator is tiled: within each (head, 128-query tile) block the element
+// (query r, column c) sits at (c / 4) * 512 + r * 4 + c % 4, so that one warp
+// adding four columns of 32 consecutive query rows touches 512 contiguous
+// bytes.  `sched` is the work counter of the main kernel's dynamic scheduler.
 struct Workspace {
-  size_t dq_off, d_off, l2_off, total;
+  size_t dq_off, d_off, l2_off, sched_off, total;
 };
 __host__ __device__ inline Workspace workspace_layout(int BH, int Npad, int d) {
   Workspace w;
   w.dq_off = 0;
   w.d_off = align256((size_t)BH * Npad * d * sizeof(float));
   w.l2_off = w.d_off + align256((size_t)BH * Npad * sizeof(float));
-  w.total = w.l2_off + align256((size_t)BH * Npad * sizeof(float));
+  w.sched_off = w.l2_off + align256((size_t)BH * Npad * sizeof(float));
+  w.total = w.sched_off + 256;
   return w;
 }
 
@@ -69,9 +75,10 @@ template <int D>
 __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restrict__ O,
                                                    const __nv_bfloat16* __restrict__ dO,
                                                    const float* __restrict__ LSE, float* __restrict__ Dw,
-                                                   float* __restrict__ L2w, float* __restrict__ dq_acc, int BH, int N,
-                                                   int Npad) {
+                                                   float* __restrict__ L2w, float* __restrict__ dq_acc,
+                                                   uint32_t* __restrict__ sched, int BH, int N, int Npad) {
   constexpr int LPR = D / 8;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0u;
   constexpr int RPW = 32 / LPR;
   const int lane = threadIdx.x & 31;
   const int sub = lane / LPR, li = lane % LPR;
@@ -116,24 +123,32 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restri
 }
 
 // --------------------------------------------------------------- convert ---
+// Thread g handles 8 columns of one query row; consecutive threads take
+// consecutive rows so the reads of the tiled accumulator are contiguous.
 template <int D>
 __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict__ dq_acc,
                                                          __nv_bfloat16* __restrict__ dQ, int BH, int N, int Npad,
                                                          float scale) {
-  const long long total = (long long)BH * N * (D / 8);
+  constexpr int PER_TILE = 128 * (D / 8);
+  const int nq = Npad / 128;
+  const long long total = (long long)BH * nq * PER_TILE;
   for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < total;
        g += (long long)gridDim.x * blockDim.x) {
-    const long long row = g / (D / 8);
-    const int c8 = (int)(g % (D / 8)) * 8;
-    const int bh = (int)(row / N), n = (int)(row % N);
-    const float4* s = reinterpret_cast<const float4*>(dq_acc + ((size_t)bh * Npad + n) * D + c8);
-    const float4 a = s[0], b = s[1];
+    const long long tile = g / PER_TILE;  // bh * nq + qt
+    const int rem = (int)(g % PER_TILE);
+    const int e2 = rem / 128, r = rem % 128;
+    const int bh = (int)(tile / nq), qt = (int)(tile % nq);
+    const int n = qt * 128 + r;
+    if (n >= N) continue;
+    const float* t = dq_acc + (size_t)tile * 128 * D;
+    const float4 a = *reinterpret_cast<const float4*>(t + (2 * e2) * 512 + r * 4);
+    const float4 b = *reinterpret_cast<const float4*>(t + (2 * e2 + 1) * 512 + r * 4);
     uint4 o;
     o.x = pack_bf16x2(a.x * scale, a.y * scale);
     o.y = pack_bf16x2(a.z * scale, a.w * scale);
     o.z = pack_bf16x2(b.x * scale, b.y * scale);
     o.w = pack_bf16x2(b.z * scale, b.w * scale);
-    *reinterpret_cast<uint4*>(dQ + (size_t)row * D + c8) = o;
+    *reinterpret_cast<uint4*>(dQ + ((size_t)bh * N + n) * D + 8 * e2) = o;
   }
 }
 
@@ -149,8 +164,14 @@ struct Cfg {
   static constexpr int OFF_DS = 2 * TILE_BYTES;           // dS^T, 128 x 128 bf16 (2 chunks)
   static constexpr int OFF_QD = 2 * TILE_BYTES + 32768;   // stages of (Q, dO)
   static constexpr int SMEM_BYTES = OFF_QD + NST * 2 * TILE_BYTES + 1024;
-  static constexpr int COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
-  static constexpr int NDQ = D == 64 ? 2 : 1;  // dQ buffers in tensor memory
+  // Tensor memory columns.  S^T fp32 in [0,128); once read, P^T (bf16) goes
+  // to [0,64) and dS^T (bf16) to [64,128).  dP^T fp32 in [128,256).
+  static constexpr int COL_S = 0, COL_P = 0, COL_DS = 64, COL_DP = 128;
+  static constexpr int COL_DV = 256, COL_DK = 256 + D;
+  // dQ: d = 128 reuses the dP^T columns once dS is formed (one buffer);
+  // d = 64 has two spare 64-column buffers after dK.
+  static constexpr int NDQ = D == 64 ? 2 : 1;
+  __host__ __device__ static constexpr int col_dq(int b) { return D == 128 ? 128 : 384 + 64 * b; }
 };
 
 struct Params {
@@ -160,6 +181,8 @@ struct Params {
   const float* Dw;
   const float* L2w;
   float* dq_acc;
+  uint32_t* sched;
+  int group;  // heads per scheduling group
   __nv_bfloat16* dK;
   __nv_bfloat16* dV;
   uint64_t timeout_ns;
@@ -170,14 +193,22 @@ struct Item {
   int bh, j;
 };
 
-// Work item idx -> (head, key tile); low key tiles first: under a causal
-// mask they meet the most query tiles.
+// Work item idx -> (head, key tile).  Heads are taken in groups of
+// p.group, so the query-side tiles and dQ rows in flight at any time belong
+// to a few heads and stay in L2; within a group low key tiles come first
+// (under a causal mask they meet the most query tiles and run longest).
 __device__ __forceinline__ Item item_at(const Params& p, int idx) {
+  const int per_group = p.group * p.nq;
+  const int g = idx / per_group, r = idx % per_group;
+  const int gsize = min(p.group, p.BH - g * p.group);
   Item it;
-  it.j = idx / p.BH;
-  it.bh = idx % p.BH;
+  it.j = r / gsize;
+  it.bh = g * p.group + r % gsize;
   return it;
 }
+
+constexpr int RING = 4;     // depth of the item ring the producer fills
+constexpr int CONSUMERS = 13;  // MMA warp + 8 softmax warps + 4 drain warps
 
 // Next query tile >= i that attends to key tile j (nq if none).
 __device__ __forceinline__ int next_q(const Params& p, int j, int i) {
@@ -198,6 +229,10 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
+// Register budget: the launch gives 128 per thread (512 threads); the
+// producer/MMA warpgroup needs few, the softmax and dQ-drain warpgroups more.
+// 128 threads x (88 + 136 + 136 + 136) = 63488 <= 65536, the launch total.
+
 template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
@@ -207,12 +242,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-  __shared__ __align__(8) uint64_t kv_full, kv_empty, s_full, p_full, ds_full, dkdv_full, mma_drain;
-  // The two column halves of a lane quarter write their packed bf16 results
-  // into columns the other half may still be reading as fp32: each half
-  // arrives once its loads are done and waits for the other before storing.
-  __shared__ __align__(8) uint64_t s_read, dp_read;
+  __shared__ __align__(8) uint64_t kv_full, kv_empty, s_full, dp_full, p_full, ds_full, dkdv_full, mma_drain;
+  // The two column halves of a lane quarter write packed bf16 results into
+  // columns the other half may still be reading as fp32 scores: each half
+  // arrives once its score loads are done and waits for the other before
+  // storing.
+  __shared__ __align__(8) uint64_t s_read;
   __shared__ __align__(8) uint64_t qd_full[C::NST], qd_empty[C::NST], dq_full[C::NDQ], dq_free[C::NDQ];
+  // Dynamic schedule: the producer claims work items from a global counter
+  // and passes them to the other roles through this ring.
+  __shared__ __align__(8) uint64_t item_full[RING], item_empty[RING];
+  __shared__ int item_ring[RING];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -222,12 +262,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(&kv_full, 1);
     mbar_init(&kv_empty, 1);
     mbar_init(&s_full, 1);
+    mbar_init(&dp_full, 1);
     mbar_init(&p_full, 256);
     mbar_init(&ds_full, 256);
     mbar_init(&dkdv_full, 1);
     mbar_init(&mma_drain, 1);
     mbar_init(&s_read, 256);
-    mbar_init(&dp_read, 256);
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(&qd_full[s], 1);
       mbar_init(&qd_empty[s], 1);
@@ -235,6 +275,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int b = 0; b < C::NDQ; ++b) {
       mbar_init(&dq_full[b], 1);
       mbar_init(&dq_free[b], 128);
+    }
+    for (int r = 0; r < RING; ++r) {
+      mbar_init(&item_full[r], 1);
+      mbar_init(&item_empty[r], CONSUMERS);
     }
     fence_barrier_init();
   }
@@ -259,12 +303,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sDS = smem + C::OFF_DS;
   uint8_t* sQD = smem + C::OFF_QD;
 
+  // Consumer side of the item ring: the k-th item this CTA processes.
+  auto take_item = [&](uint32_t k, int& idx) -> bool {
+    const uint32_t slot = k % RING;
+    if (!mbar_wait(&item_full[slot], (k / RING) & 1, w)) return false;
+    idx = *reinterpret_cast<volatile int*>(&item_ring[slot]);
+    mbar_arrive(&item_empty[slot]);
+    return true;
+  };
+  auto take_item_warp = [&](uint32_t k, int& idx) -> bool {
+    const uint32_t slot = k % RING;
+    if (!mbar_wait_warp(&item_full[slot], (k / RING) & 1, w)) return false;
+    idx = *reinterpret_cast<volatile int*>(&item_ring[slot]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&item_empty[slot]);
+    return true;
+  };
+
+  if (warp < 4) {
+    regs_dec<88>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t item_iter = 0, qd_iter = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_iter) {
+      for (;; ++item_iter) {
+        const uint32_t slot = item_iter % RING;
+        ok = mbar_wait(&item_empty[slot], ((item_iter / RING) & 1) ^ 1, w);
+        if (!ok) break;
+        int idx = (int)atomicAdd(p.sched, 1u);
+        if (idx > p.n_items) idx = p.n_items;
+        item_ring[slot] = idx;
+        mbar_arrive(&item_full[slot]);
+        if (idx >= p.n_items) break;
         const Item it = item_at(p, idx);
         ok = mbar_wait(&kv_empty, (item_iter & 1) ^ 1, w);
         if (!ok) break;
@@ -301,43 +372,64 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC_T = idesc_bf16_f32(128, 128, 0, 0);   // S^T, dP^T: K-major A and B
-      constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, 0, 1);     // dV, dK: A in TMEM, B MN-major
-      constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, 64, 1, 1);    // dQ (64-column pieces): both MN-major
+      constexpr uint32_t IDESC_T = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T: K-major A and B
+      constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, 0, 1);    // dV, dK: A in TMEM, B MN-major
+      constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, 1, 1);    // dQ: both MN-major
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aDS = smem_u32(sDS), aQD = smem_u32(sQD);
       uint32_t item_iter = 0, qd_iter = 0, dq_iter = 0, p_cnt = 0, ds_cnt = 0;
       bool ok = true, issued = false;
-      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_iter) {
+
+      // S^T = K Q^T into the score columns (M = keys, N = queries, K = d).
+      auto issue_s = [&](uint32_t st) {
+        const uint32_t aQ = aQD + st * 2 * C::TILE_BYTES;
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s) {
+          const uint32_t off = (s >> 2) * C::CHUNK_BYTES + (s & 3) * 32;
+          mma_ss(tmem + C::COL_S, smem_desc_sw128(aK + off, 16, 1024), smem_desc_sw128(aQ + off, 16, 1024),
+                 IDESC_T, s > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full);
+      };
+      // dP^T = V dO^T.  With d = 128 the dP^T columns hold the previous dQ
+      // tile until the drain warps have read it.
+      auto issue_dp = [&](uint32_t st) -> bool {
+        if (D == 128 && dq_iter > 0) {
+          if (!mbar_wait(&dq_free[0], (dq_iter - 1) & 1, w)) return false;
+          tc_fence_after();
+        }
+        const uint32_t adO = aQD + st * 2 * C::TILE_BYTES + C::TILE_BYTES;
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s) {
+          const uint32_t off = (s >> 2) * C::CHUNK_BYTES + (s & 3) * 32;
+          mma_ss(tmem + C::COL_DP, smem_desc_sw128(aV + off, 16, 1024), smem_desc_sw128(adO + off, 16, 1024),
+                 IDESC_T, s > 0 ? 1u : 0u);
+        }
+        tc_commit(&dp_full);
+        return true;
+      };
+
+      for (;; ++item_iter) {
+        int idx;
+        ok = take_item(item_iter, idx);
+        if (!ok || idx >= p.n_items) break;
         const Item it = item_at(p, idx);
         ok = mbar_wait(&kv_full, item_iter & 1, w);
         if (!ok) break;
-        int n = 0;
-        for (int i = next_q(p, it.j, 0); ok && i < p.nq; i = next_q(p, it.j, i + 1), ++n) {
-          const uint32_t st = qd_iter % C::NST;
-          const uint32_t b = dq_iter % C::NDQ;
-          ok = mbar_wait(&qd_full[st], (qd_iter / C::NST) & 1, w);
-          // The dQ buffer about to be written must have been drained.  For
-          // d = 128 it overlaps the S^T / dP^T columns, so wait before those.
-          if (ok && dq_iter >= (uint32_t)C::NDQ) ok = mbar_wait(&dq_free[b], ((dq_iter / C::NDQ) - 1) & 1, w);
+        int i = next_q(p, it.j, 0);
+        if (i < p.nq) {
+          ok = mbar_wait(&qd_full[qd_iter % C::NST], (qd_iter / C::NST) & 1, w);
           if (!ok) break;
           tc_fence_after();
+          issue_s(qd_iter % C::NST);
+          issued = true;
+          ok = issue_dp(qd_iter % C::NST);
+          if (!ok) break;
+        }
+        for (int n = 0; ok && i < p.nq; ++n) {
+          const int inext = next_q(p, it.j, i + 1);
+          const uint32_t st = qd_iter % C::NST;
           const uint32_t aQ = aQD + st * 2 * C::TILE_BYTES;
           const uint32_t adO = aQ + C::TILE_BYTES;
-          // S^T = K Q^T and dP^T = V dO^T (M = keys, N = queries, K = d)
-#pragma unroll
-          for (int s = 0; s < D / 16; ++s) {
-            const uint32_t off = (s >> 2) * C::CHUNK_BYTES + (s & 3) * 32;
-            mma_ss(tmem + C::COL_S, smem_desc_sw128(aK + off, 16, 1024), smem_desc_sw128(aQ + off, 16, 1024),
-                   IDESC_T, s > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int s = 0; s < D / 16; ++s) {
-            const uint32_t off = (s >> 2) * C::CHUNK_BYTES + (s & 3) * 32;
-            mma_ss(tmem + C::COL_DP, smem_desc_sw128(aV + off, 16, 1024), smem_desc_sw128(adO + off, 16, 1024),
-                   IDESC_T, s > 0 ? 1u : 0u);
-          }
-          tc_commit(&s_full);
-          issued = true;
           // dV += P^T dO (A = P^T in TMEM, K = 128 queries)
           ok = mbar_wait(&p_full, p_cnt & 1, w);
           if (!ok) break;
@@ -345,7 +437,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
 #pragma unroll
           for (int s = 0; s < BQ / 16; ++s)
-            mma_ts(tmem + C::COL_DV, tmem + C::COL_S + s * 8, smem_desc_sw128(adO + s * 2048, C::CHUNK_BYTES, 1024),
+            mma_ts(tmem + C::COL_DV, tmem + C::COL_P + s * 8, smem_desc_sw128(adO + s * 2048, C::CHUNK_BYTES, 1024),
                    IDESC_G, (n > 0 || s > 0) ? 1u : 0u);
           // dK += dS^T Q; dQ_i = dS K
           ok = mbar_wait(&ds_full, ds_cnt & 1, w);
@@ -354,21 +446,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
 #pragma unroll
           for (int s = 0; s < BQ / 16; ++s)
-            mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + s * 8, smem_desc_sw128(aQ + s * 2048, C::CHUNK_BYTES, 1024),
+            mma_ts(tmem + C::COL_DK, tmem + C::COL_DS + s * 8, smem_desc_sw128(aQ + s * 2048, C::CHUNK_BYTES, 1024),
                    IDESC_G, (n > 0 || s > 0) ? 1u : 0u);
-#pragma unroll
-          for (int h = 0; h < D / 64; ++h) {
-            const uint32_t col = D == 128 ? (h == 0 ? 64u : 192u) : (384u + 64u * b);
-#pragma unroll
-            for (int s = 0; s < BK / 16; ++s)
-              mma_ss(tmem + col, smem_desc_sw128(aDS + s * 2048, C::CHUNK_BYTES, 1024),
-                     smem_desc_sw128(aK + h * C::CHUNK_BYTES + s * 2048, C::CHUNK_BYTES, 1024), IDESC_Q,
-                     s > 0 ? 1u : 0u);
+          const uint32_t b = dq_iter % C::NDQ;
+          if (D == 64 && dq_iter >= (uint32_t)C::NDQ) {
+            ok = mbar_wait(&dq_free[b], ((dq_iter / C::NDQ) - 1) & 1, w);
+            if (!ok) break;
+            tc_fence_after();
           }
+#pragma unroll
+          for (int s = 0; s < BK / 16; ++s)
+            mma_ss(tmem + C::col_dq(b), smem_desc_sw128(aDS + s * 2048, C::CHUNK_BYTES, 1024),
+                   smem_desc_sw128(aK + s * 2048, C::CHUNK_BYTES, 1024), IDESC_Q, s > 0 ? 1u : 0u);
           tc_commit(&dq_full[b]);
           tc_commit(&qd_empty[st]);
           ++qd_iter;
           ++dq_iter;
+          // Start the next query tile: S^T does not depend on the dQ drain.
+          if (inext < p.nq) {
+            const uint32_t stn = qd_iter % C::NST;
+            ok = mbar_wait(&qd_full[stn], (qd_iter / C::NST) & 1, w);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(stn);
+            ok = issue_dp(stn);
+          }
+          i = inext;
         }
         if (!ok) break;
         tc_commit(&dkdv_full);
@@ -379,7 +482,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_drain_wait(&mma_drain, 0, globaltimer_ns() + 100000000ull);
       }
     }
-  } else if (warp >= 4 && warp < 12) {
+  }
+  } else if (warp < 12) {
+    regs_inc<136>();
     // ------------------------------------------------------------ softmax
     const int quarter = warp & 3;
     const int hf = (warp - 4) >> 2;        // query half: columns [64 hf, 64 hf + 64)
@@ -388,19 +493,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const float sl2 = p.scale_log2;
     uint32_t s_cnt = 0, dk_cnt = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x) {
+    for (uint32_t k = 0;; ++k) {
+      int idx;
+      ok = take_item_warp(k, idx);
+      if (!ok || idx >= p.n_items) break;
       const Item it = item_at(p, idx);
       const int key = it.j * BK + kr;
       bool any = false;
       for (int i = next_q(p, it.j, 0); i < p.nq; i = next_q(p, it.j, i + 1)) {
         ok = mbar_wait_warp(&s_full, s_cnt & 1, w);
         if (!ok) break;
+        const uint32_t par = s_cnt & 1;
         ++s_cnt;
         tc_fence_after();
         const int q0 = i * BQ + hf * 64;  // first query of this thread's half
         const size_t rowbase = (size_t)it.bh * p.Npad + q0;
         const bool key_live = key < p.N;
         const bool diag = p.mask_kind == FA_MASK_CAUSAL && i == it.j;
+        // ---- P^T = exp2(S^T * scale * log2e - LSE_i * log2e)
         float pr[64];
         {
           uint32_t sr[64];
@@ -427,26 +537,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
-          ok = mbar_wait_warp(&s_read, (s_cnt - 1) & 1, w);
+          ok = mbar_wait_warp(&s_read, par, w);
           if (!ok) break;
           tc_fence_after();
-          FA_TMEM_ST_X32(tmem + lane_bits + C::COL_S + hf * 32, pk);
+          FA_TMEM_ST_X32(tmem + lane_bits + C::COL_P + hf * 32, pk);
         }
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full);
-        // dS^T = P^T * (dP^T - D)
-        uint8_t* ds_chunk = sDS + hf * C::CHUNK_BYTES + kr * 128;
+        // ---- dS^T = P^T * (dP^T - D)
+        ok = mbar_wait_warp(&dp_full, par, w);
+        if (!ok) break;
+        tc_fence_after();
         uint32_t dk[32];
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           uint32_t dr[32];
           FA_TMEM_LD_X32(tmem + lane_bits + C::COL_DP + hf * 64 + cc * 32, dr);
           tc_wait_ld();
-          if (cc == 1) {
-            tc_fence_before();
-            mbar_arrive(&dp_read);
-          }
           const float4* d4 = reinterpret_cast<const float4*>(p.Dw + rowbase + cc * 32);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -460,18 +568,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             dk[cc * 16 + u * 2 + 1] = pack_bf16x2(g2, g3);
           }
         }
-        // shared-memory copy of dS^T, 128-byte swizzle: 16-byte unit u of
-        // row kr lives at unit (u ^ (kr & 7)).
+        // Shared-memory copy of dS^T (the A operand of dQ = dS K), 128-byte
+        // swizzle: 16-byte unit u of row kr lives at unit (u ^ (kr & 7)).
+        uint8_t* ds_row = sDS + hf * C::CHUNK_BYTES + kr * 128;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int unit = u ^ (kr & 7);
-          *reinterpret_cast<uint4*>(ds_chunk + unit * 16) =
-              make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+          *reinterpret_cast<uint4*>(ds_row + unit * 16) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
         }
-        ok = mbar_wait_warp(&dp_read, (s_cnt - 1) & 1, w);
-        if (!ok) break;
-        tc_fence_after();
-        FA_TMEM_ST_X32(tmem + lane_bits + C::COL_DP + hf * 32, dk);
+        FA_TMEM_ST_X32(tmem + lane_bits + C::COL_DS + hf * 32, dk);
         tc_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
@@ -509,38 +614,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_before();
     }
-  } else if (warp >= 12) {
+  } else {
+    regs_inc<136>();
     // ------------------------------------------------------------ dQ drain
+    // Read the whole dQ tile row out of tensor memory, hand the columns back
+    // to the MMA warp, then add the row into the fp32 accumulator.
     const int quarter = warp & 3;
     const int qr = quarter * 32 + lane;
     const uint32_t lane_bits = uint32_t(quarter * 32) << 16;
     uint32_t dq_iter = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x) {
+    for (uint32_t k = 0;; ++k) {
+      int idx;
+      ok = take_item_warp(k, idx);
+      if (!ok || idx >= p.n_items) break;
       const Item it = item_at(p, idx);
       for (int i = next_q(p, it.j, 0); i < p.nq; i = next_q(p, it.j, i + 1)) {
         const uint32_t b = dq_iter % C::NDQ;
         ok = mbar_wait_warp(&dq_full[b], (dq_iter / C::NDQ) & 1, w);
         if (!ok) break;
         tc_fence_after();
-        float* dst = p.dq_acc + ((size_t)it.bh * p.Npad + (size_t)i * BQ + qr) * D;
+        uint32_t v[D];
 #pragma unroll
-        for (int h = 0; h < D / 64; ++h) {
-          const uint32_t col = D == 128 ? (h == 0 ? 64u : 192u) : (384u + 64u * b);
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            uint32_t v[32];
-            FA_TMEM_LD_X32(tmem + lane_bits + col + cc * 32, v);
-            tc_wait_ld();
-            float* d = dst + h * 64 + cc * 32;
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              red_add_v4(d + 4 * e, __uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                         __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
-          }
-        }
+        for (int c = 0; c < D; c += 32) FA_TMEM_LD_X32(tmem + lane_bits + C::col_dq(b) + c, (v + c));
+        tc_wait_ld();
         tc_fence_before();
         mbar_arrive(&dq_free[b]);
+        // tiled accumulator: columns 4e..4e+3 of row qr at e * 512 + qr * 4
+        float* dst = p.dq_acc + ((size_t)it.bh * p.Npad + (size_t)i * BQ) * D + qr * 4;
+#pragma unroll
+        for (int e = 0; e < D / 4; ++e)
+          red_add_v4(dst + e * 512, __uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                     __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
         ++dq_iter;
       }
     }
@@ -572,6 +677,7 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
   float* dq_acc = reinterpret_cast<float*>(ws + wl.dq_off);
   float* Dw = reinterpret_cast<float*>(ws + wl.d_off);
   float* L2w = reinterpret_cast<float*>(ws + wl.l2_off);
+  uint32_t* sched = reinterpret_cast<uint32_t*>(ws + wl.sched_off);
   const int sms = num_sms();
 
   if (stage < 0 || stage == 0) {
@@ -581,7 +687,7 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
     bwd::prep_kernel<D><<<(int)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(O),
                                                      static_cast<const __nv_bfloat16*>(dO), LSE, Dw, L2w, dq_acc,
-                                                     pr.BH, pr.N, Npad);
+                                                     sched, pr.BH, pr.N, Npad);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stage < 0 || stage == 1) {
@@ -598,6 +704,8 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     p.Dw = Dw;
     p.L2w = L2w;
     p.dq_acc = dq_acc;
+    p.sched = sched;
+    p.group = pr.BH < 8 ? pr.BH : 8;
     p.dK = static_cast<__nv_bfloat16*>(dK);
     p.dV = static_cast<__nv_bfloat16*>(dV);
     p.timeout_ns = wait_timeout_ns();
@@ -610,7 +718,7 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stage < 0 || stage == 2) {
-    const long long work = (long long)pr.BH * pr.N * (D / 8);
+    const long long work = (long long)pr.BH * Npad * (D / 8);
     long long blocks = (work + 255) / 256;
     if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
     bwd::dq_convert_kernel<D><<<(int)blocks, 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), pr.BH, pr.N,

@@ -53,6 +53,7 @@ struct Cfg {
 
 struct Params {
   int BH, N, nq, n_pairs, n_items, mask_kind;
+  int group;  // heads per scheduling group
   const uint8_t* block_mask;
   float scale_log2;
   __nv_bfloat16* O;
@@ -66,12 +67,17 @@ struct Item {
   bool has1;
 };
 
-// Work item idx -> (head, pair of query tiles).  Later query tiles come first
-// so that, under a causal mask, the longest items start earliest.
+// Work item idx -> (head, pair of query tiles).  Heads are taken in groups
+// of p.group so that the K/V tiles in flight belong to a few heads and stay
+// in L2; within a group later query tiles come first, so that under a causal
+// mask the longest items start earliest.
 __device__ __forceinline__ Item item_at(const Params& p, int idx) {
   Item it;
-  const int c = p.n_pairs - 1 - idx / p.BH;
-  it.bh = idx % p.BH;
+  const int per_group = p.group * p.n_pairs;
+  const int g = idx / per_group, r = idx % per_group;
+  const int gsize = min(p.group, p.BH - g * p.group);
+  const int c = p.n_pairs - 1 - r / gsize;
+  it.bh = g * p.group + r % gsize;
   it.q0 = 2 * c;
   it.q1 = 2 * c + 1;
   it.has1 = it.q1 < p.nq;
@@ -149,6 +155,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = tmem_base_sh;
   const WaitCtx w{p.timeout_ns, &abort_flag, p.status};
 
+  // Registers: 384 threads x 168 at launch; the producer/MMA warpgroup gives
+  // much of its share to the two softmax warpgroups: 128 x (88 + 208 + 208)
+  // = 64512, the launch total.
+  if (warp < 4) {
+    regs_dec<88>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -293,7 +304,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_drain_wait(&mma_drain, 0, globaltimer_ns() + 100000000ull);
       }
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_inc<208>();
     // ------------------------------------------------------------ softmax
     const int t = (warp - 4) >> 2;         // query tile of this warpgroup
     const int quarter = warp & 3;          // tensor-memory lane quarter
@@ -436,6 +449,7 @@ fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void
   p.nq = pr.nq;
   p.n_pairs = (pr.nq + 1) / 2;
   p.n_items = p.n_pairs * pr.BH;
+  p.group = pr.BH < 8 ? pr.BH : 8;
   p.mask_kind = pr.mask_kind;
   p.block_mask = pr.block_mask;
   p.scale_log2 = pr.scale_log2;
