@@ -170,6 +170,23 @@ def reference_arm(args, w):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(v: float, dist=None, device=None) -> float:
+    """Largest value of `v` over all ranks (the step time that counts)."""
+    if dist is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(total_ms: float, steps: int, world: int, flops_per_step: float) -> tuple:
+    """(ms per step, whole-job TFLOP/s): every rank runs one replica of the
+    workload, so the job does `world` replicas per step in the slowest rank's
+    time."""
+    ms = total_ms / steps
+    return ms, world * flops_per_step / (ms * 1e-3) / 1e12
+
+
 def workload_config(w):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "mask": w.mask, "scale": w.scale}
 
@@ -208,13 +225,6 @@ def main():
     def barrier():
         if dist is not None:
             dist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if dist is None:
-            return v
-        t = torch.tensor([v], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # ---- inputs resident in HBM (each rank its own replica of the workload)
     x = workloads.make_inputs(w, args.seed + rank)
@@ -259,13 +269,12 @@ def main():
     barrier()
     clocks.mark_end()
     status = fa.device_status()
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
     per_kernel = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(names)}
     clock_info = clocks.result()
 
     fl = flops(w, mask_cpu)
-    ms_step = total_ms / args.steps
-    value = world * (fl["fwd"] + fl["bwd"]) / (ms_step * 1e-3) / 1e12
+    ms_step, value = throughput(total_ms, args.steps, world, fl["fwd"] + fl["bwd"])
     peaks, peak_kind = load_peaks()
     fwd_tflops = fl["fwd"] / (per_kernel["fwd"] * 1e-3) / 1e12
     bwd_ms = per_kernel["bwd_prep"] + per_kernel["bwd_main"] + per_kernel["bwd_dq_convert"]
@@ -319,8 +328,8 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
-    e2e_value = world * (fl["fwd"] + fl["bwd"]) / (e2e_ms * 1e-3) / 1e12
+    e2e_ms, e2e_value = throughput(max_over_ranks(e0.elapsed_time(e1), dist, dev), e2e_steps, world,
+                                   fl["fwd"] + fl["bwd"])
     status = status or fa.device_status()
 
     cpu = None
