@@ -35,6 +35,8 @@ SIGNATURES = {
     "fa_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fa_bwd_stage": (_i, [_i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp, _vp,
                           _sz, _vp]),
+    "fa_bwd_static_workspace": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp,
+                                     _vp, _vp]),
     "fa_device_status": (_i, [_vp]),
     "fa_set_wait_timeout_ns": (None, [_u64]),
     "fa_status_string": (ctypes.c_char_p, [_i]),

@@ -103,6 +103,35 @@ fa_status fa_bwd_stage(int stage, const void* Q, const void* K, const void* V, c
                        const uint8_t* block_mask, float scale, void* dQ, void* dK, void* dV,
                        void* workspace, size_t workspace_bytes, void* stream);
 
+/* Largest scratch, in bytes, that fa_bwd_static_workspace() can use: 64 MiB. */
+#define FA_BWD_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
+
+/* fa_bwd without a caller-supplied workspace, for callers that cannot
+ * allocate device memory: for example a runtime whose device memory is all
+ * handed out up front by its own pool, so one more cudaMalloc would fail or
+ * fragment it, or a latency-critical loop where cudaMalloc/cudaFree would
+ * stall on an implicit device synchronisation.  This call allocates nothing.
+ * Its scratch is a fixed 64 MiB array (FA_BWD_STATIC_WORKSPACE_BYTES) in the
+ * library's own device memory; every GPU that loads the library holds it
+ * until the process exits.  The paper has no counterpart to this call.
+ *   - Arguments, outputs and results are those of fa_bwd, minus the
+ *     workspace.  A problem whose fa_bwd_workspace_size() exceeds the array
+ *     is refused with FA_ERR_WORKSPACE before anything runs (that allows
+ *     B*H*ceil(N/128)*128 up to about 129,000 for d = 128 and about 254,000
+ *     for d = 64).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture begins.
+ *   - All calls on a device share the one array, and it keeps whatever the
+ *     last call left in it (each call clears what must start at zero).  Calls
+ *     whose kernels overlap on the GPU -- on different streams, or from
+ *     different host threads -- race on it and give wrong results: order
+ *     them on one stream or synchronise between them. */
+fa_status fa_bwd_static_workspace(const void* Q, const void* K, const void* V, const void* O,
+                                  const void* dO, const float* LSE, int B, int H, int N, int d,
+                                  int mask_kind, const uint8_t* block_mask, float scale, void* dQ,
+                                  void* dK, void* dV, void* stream);
+
 /* Synchronise `stream`, then read and clear the calling device's status
  * word.  Returns FA_OK, FA_ERR_TIMEOUT if a bounded wait ran out in a kernel
  * since the last call, or FA_ERR_CUDA if the synchronisation itself failed. */
