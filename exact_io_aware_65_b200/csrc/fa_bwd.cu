@@ -163,7 +163,13 @@ struct Cfg {
   static constexpr int OFF_V = TILE_BYTES;
   static constexpr int OFF_DS = 2 * TILE_BYTES;           // dS^T, 128 x 128 bf16 (2 chunks)
   static constexpr int OFF_QD = 2 * TILE_BYTES + 32768;   // stages of (Q, dO)
-  static constexpr int SMEM_BYTES = OFF_QD + NST * 2 * TILE_BYTES + 1024;
+  // Per stage: the 128 LSE*log2(e) values then the 128 D values of the
+  // stage's query tile (fp32, 1 KB).
+  static constexpr int OFF_LD = OFF_QD + NST * 2 * TILE_BYTES;
+  // The dynamic region starts 1024-byte aligned (the extern declaration
+  // asks for it), so no slack is added: at d = 128 this is 226 KB, which
+  // with the static barriers fills the 227 KB a CTA may use.
+  static constexpr int SMEM_BYTES = OFF_LD + NST * 1024;
   // Tensor memory columns.  S^T fp32 in [0,128); once read, P^T (bf16) goes
   // to [0,64) and dS^T (bf16) to [64,128).  dP^T fp32 in [128,256).
   static constexpr int COL_S = 0, COL_P = 0, COL_DS = 64, COL_DP = 128;
@@ -239,8 +245,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapdO,
                 const Params p) {
   using C = Cfg<D>;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
 
   __shared__ __align__(8) uint64_t kv_full, kv_empty, s_full, dp_full, p_full, ds_full, dkdv_full, mma_drain;
   // The two column halves of a lane quarter write packed bf16 results into
@@ -302,6 +307,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sV = smem + C::OFF_V;
   uint8_t* sDS = smem + C::OFF_DS;
   uint8_t* sQD = smem + C::OFF_QD;
+  const float* sLD = reinterpret_cast<const float*>(smem + C::OFF_LD);
 
   // Consumer side of the item ring: the k-th item this CTA processes.
   auto take_item = [&](uint32_t k, int& idx) -> bool {
@@ -349,13 +355,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t st = qd_iter % C::NST;
           ok = mbar_wait(&qd_empty[st], ((qd_iter / C::NST) & 1) ^ 1, w);
           if (!ok) break;
-          mbar_arrive_expect_tx(&qd_full[st], 2 * C::TILE_BYTES);
+          mbar_arrive_expect_tx(&qd_full[st], 2 * C::TILE_BYTES + 1024);
           uint8_t* q = sQD + st * 2 * C::TILE_BYTES;
 #pragma unroll
           for (int c = 0; c < C::CHUNKS; ++c) {
             tma_load_3d(q + c * C::CHUNK_BYTES, &mapQ, &qd_full[st], c * 64, i * BQ, it.bh);
             tma_load_3d(q + C::TILE_BYTES + c * C::CHUNK_BYTES, &mapdO, &qd_full[st], c * 64, i * BQ, it.bh);
           }
+          const size_t row0 = (size_t)it.bh * p.Npad + (size_t)i * BQ;
+          uint8_t* ld = smem + C::OFF_LD + st * 1024;
+          bulk_load(ld, p.L2w + row0, 512, &qd_full[st]);
+          bulk_load(ld + 512, p.Dw + row0, 512, &qd_full[st]);
           ++qd_iter;
         }
       }
@@ -506,8 +516,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t par = s_cnt & 1;
         ++s_cnt;
         tc_fence_after();
-        const int q0 = i * BQ + hf * 64;  // first query of this thread's half
-        const size_t rowbase = (size_t)it.bh * p.Npad + q0;
+        // this query tile's LSE and D values, staged in shared memory by the
+        // producer with Q and dO (same stage index as the MMA warp uses)
+        const float* sL = sLD + ((s_cnt - 1) % C::NST) * 256 + hf * 64;
+        const float* sD = sL + 128;
         const bool key_live = key < p.N;
         const bool diag = p.mask_kind == FA_MASK_CAUSAL && i == it.j;
         // ---- P^T = exp2(S^T * scale * log2e - LSE_i * log2e)
@@ -519,10 +531,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_wait_ld();
           tc_fence_before();
           mbar_arrive(&s_read);
-          const float4* l4 = reinterpret_cast<const float4*>(p.L2w + rowbase);
+          const float4* l4 = reinterpret_cast<const float4*>(sL);
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
-            const float4 lv = __ldg(l4 + u);
+            const float4 lv = l4[u];
             const float lvv[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -555,10 +567,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t dr[32];
           FA_TMEM_LD_X32(tmem + lane_bits + C::COL_DP + hf * 64 + cc * 32, dr);
           tc_wait_ld();
-          const float4* d4 = reinterpret_cast<const float4*>(p.Dw + rowbase + cc * 32);
+          const float4* d4 = reinterpret_cast<const float4*>(sD + cc * 32);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const float4 dv = __ldg(d4 + u);
+            const float4 dv = d4[u];
             const int c = cc * 32 + u * 4;
             const float g0 = pr[c + 0] * (__uint_as_float(dr[u * 4 + 0]) - dv.x);
             const float g1 = pr[c + 1] * (__uint_as_float(dr[u * 4 + 1]) - dv.y);

@@ -348,9 +348,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int c = 0; c < BN; ++c)
             if (c >= lim) x[c] = -INFINITY;
         }
-        float mx = x[0];
+        // row max as eight independent chains, then a tree
+        float ma[8];
 #pragma unroll
-        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, x[c]);
+        for (int k = 0; k < 8; ++k) ma[k] = x[k];
+#pragma unroll
+        for (int c = 8; c < BN; c += 8)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) ma[k] = fmaxf(ma[k], x[c + k]);
+        float mx = fmaxf(fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3])), fmaxf(fmaxf(ma[4], ma[5]), fmaxf(ma[6], ma[7])));
         mx *= sl2;
         const bool grow = mx > m + RESCALE_THRESHOLD;
         float alpha = 1.0f;
@@ -377,7 +383,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         first = false;
         const float m_use = (m == -INFINITY) ? 0.0f : m;
-        float rs = 0.0f;
+        float rsa[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // row sum, eight chains
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t pk[32];
@@ -385,12 +391,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int i = 0; i < 32; ++i) {
             const float p0 = ex2_approx(fmaf(x[64 * h + 2 * i], sl2, -m_use));
             const float p1 = ex2_approx(fmaf(x[64 * h + 2 * i + 1], sl2, -m_use));
-            rs += p0 + p1;
+            rsa[(2 * i) & 7] += p0;
+            rsa[(2 * i + 1) & 7] += p1;
             pk[i] = pack_bf16x2(p0, p1);
           }
           FA_TMEM_ST_X32(t_s + 32 * h, pk);
         }
-        l += rs;
+        l += ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[t]);
