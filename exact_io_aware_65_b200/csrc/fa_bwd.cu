@@ -30,11 +30,12 @@
 // CTA roles (512 threads): warp 0 TMA producer; warp 1 MMA issuer; warps
 // 4..11 softmax (thread = key row; warps 4..7 take query columns 0..63,
 // warps 8..11 columns 64..127); warps 12..15 dQ drain (thread = query row).
-// Tensor memory: S^T [0,128), then P^T (bf16) in [0,64) and dS^T (bf16) in
-// [64,128); dP^T [128,256); dV [256, 256+d); dK [256+d, 256+2d).  The dQ
-// tile reuses the dP^T columns for d = 128 (so the next dP^T waits for the
-// drain, the next S^T does not), and has two buffers at [384,448) and
-// [448,512) for d = 64.
+// Tensor memory: S^T [0,128), then P^T (bf16) in [0,64); dP^T [128,256),
+// then dS^T (bf16) in [128,192); dV [256, 256+d); dK [256+d, 256+2d).  The
+// MMA order per query tile is dV, next S^T, dK, dQ, next dP^T, so the
+// softmax of the next tile overlaps three products.  The dQ tile reuses the
+// dP^T columns for d = 128 (the next dP^T waits for the drain) and has two
+// buffers at [384,448) and [448,512) for d = 64.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -171,11 +172,14 @@ struct Cfg {
   // with the static barriers fills the 227 KB a CTA may use.
   static constexpr int SMEM_BYTES = OFF_LD + NST * 1024;
   // Tensor memory columns.  S^T fp32 in [0,128); once read, P^T (bf16) goes
-  // to [0,64) and dS^T (bf16) to [64,128).  dP^T fp32 in [128,256).
-  static constexpr int COL_S = 0, COL_P = 0, COL_DS = 64, COL_DP = 128;
+  // to [0,64).  dP^T fp32 in [128,256); once read, dS^T (bf16) goes to
+  // [128,192).  The score columns are thus free as soon as dV has been
+  // issued, so the next tile's S^T can follow it directly.
+  static constexpr int COL_S = 0, COL_P = 0, COL_DP = 128, COL_DS = 128;
   static constexpr int COL_DV = 256, COL_DK = 256 + D;
-  // dQ: d = 128 reuses the dP^T columns once dS is formed (one buffer);
-  // d = 64 has two spare 64-column buffers after dK.
+  // dQ: d = 128 reuses the dP^T columns once dK has read dS^T (one buffer,
+  // so the next dP^T waits for the drain); d = 64 has two spare 64-column
+  // buffers after dK.
   static constexpr int NDQ = D == 64 ? 2 : 1;
   __host__ __device__ static constexpr int col_dq(int b) { return D == 128 ? 128 : 384 + 64 * b; }
 };
@@ -252,7 +256,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // columns the other half may still be reading as fp32 scores: each half
   // arrives once its score loads are done and waits for the other before
   // storing.
-  __shared__ __align__(8) uint64_t s_read;
+  __shared__ __align__(8) uint64_t s_read, dp_read;
   __shared__ __align__(8) uint64_t qd_full[C::NST], qd_empty[C::NST], dq_full[C::NDQ], dq_free[C::NDQ];
   // Dynamic schedule: the producer claims work items from a global counter
   // and passes them to the other roles through this ring.
@@ -273,6 +277,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(&dkdv_full, 1);
     mbar_init(&mma_drain, 1);
     mbar_init(&s_read, 256);
+    mbar_init(&dp_read, 256);
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(&qd_full[s], 1);
       mbar_init(&qd_empty[s], 1);
@@ -437,7 +442,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         for (int n = 0; ok && i < p.nq; ++n) {
           const int inext = next_q(p, it.j, i + 1);
-          const uint32_t st = qd_iter % C::NST;
+          const uint32_t st = qd_iter % C::NST;         // stage of query tile i
+          const uint32_t stn = (qd_iter + 1) % C::NST;  // stage of query tile inext
           const uint32_t aQ = aQD + st * 2 * C::TILE_BYTES;
           const uint32_t adO = aQ + C::TILE_BYTES;
           // dV += P^T dO (A = P^T in TMEM, K = 128 queries)
@@ -449,7 +455,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int s = 0; s < BQ / 16; ++s)
             mma_ts(tmem + C::COL_DV, tmem + C::COL_P + s * 8, smem_desc_sw128(adO + s * 2048, C::CHUNK_BYTES, 1024),
                    IDESC_G, (n > 0 || s > 0) ? 1u : 0u);
-          // dK += dS^T Q; dQ_i = dS K
+          // S^T of the next query tile goes in now: its columns were last read
+          // by the dV product just issued, and its softmax can then overlap
+          // the dK, dQ and next dP products.
+          if (inext < p.nq) {
+            ok = mbar_wait(&qd_full[stn], ((qd_iter + 1) / C::NST) & 1, w);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(stn);
+          }
+          // dK += dS^T Q (A = dS^T in TMEM); dQ_i = dS K
           ok = mbar_wait(&ds_full, ds_cnt & 1, w);
           if (!ok) break;
           ++ds_cnt;
@@ -472,15 +487,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_commit(&qd_empty[st]);
           ++qd_iter;
           ++dq_iter;
-          // Start the next query tile: S^T does not depend on the dQ drain.
-          if (inext < p.nq) {
-            const uint32_t stn = qd_iter % C::NST;
-            ok = mbar_wait(&qd_full[stn], (qd_iter / C::NST) & 1, w);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(stn);
-            ok = issue_dp(stn);
-          }
+          // dP^T of the next query tile (after the dQ drain when they share columns)
+          if (inext < p.nq) ok = issue_dp(stn);
           i = inext;
         }
         if (!ok) break;
@@ -567,6 +575,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t dr[32];
           FA_TMEM_LD_X32(tmem + lane_bits + C::COL_DP + hf * 64 + cc * 32, dr);
           tc_wait_ld();
+          if (cc == 1) {
+            tc_fence_before();
+            mbar_arrive(&dp_read);
+          }
           const float4* d4 = reinterpret_cast<const float4*>(sD + cc * 32);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -588,6 +600,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int unit = u ^ (kr & 7);
           *reinterpret_cast<uint4*>(ds_row + unit * 16) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
         }
+        // dS^T overwrites dP^T columns the other column half may still be
+        // reading: wait until both halves have loaded theirs.
+        ok = mbar_wait_warp(&dp_read, par, w);
+        if (!ok) break;
+        tc_fence_after();
         FA_TMEM_ST_X32(tmem + lane_bits + C::COL_DS + hf * 32, dk);
         tc_wait_st();
         fence_proxy_async_smem();
