@@ -182,6 +182,12 @@ struct Cfg {
   // buffers after dK.
   static constexpr int NDQ = D == 64 ? 2 : 1;
   __host__ __device__ static constexpr int col_dq(int b) { return D == 128 ? 128 : 384 + 64 * b; }
+  // How a dQ tile reaches the fp32 accumulator.  d = 64 (four Q/dO stages):
+  // staged in its own dead Q/dO stage and added with one bulk reduce-add,
+  // the stage then returned to the producer.  d = 128 (two stages): holding
+  // the stage that long would starve the producer, so each drain thread adds
+  // its row with vector reductions and the MMA warp returns the stage.
+  static constexpr bool BULK_DQ = D == 64;
 };
 
 struct Params {
@@ -207,6 +213,11 @@ struct Item {
 // p.group, so the query-side tiles and dQ rows in flight at any time belong
 // to a few heads and stay in L2; within a group low key tiles come first
 // (under a causal mask they meet the most query tiles and run longest).
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 __device__ __forceinline__ Item item_at(const Params& p, int idx) {
   const int per_group = p.group * p.nq;
   const int g = idx / per_group, r = idx % per_group;
@@ -230,14 +241,6 @@ __device__ __forceinline__ int next_q(const Params& p, int j, int i) {
   return i;
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
 
 // Register budget: the launch gives 128 per thread (512 threads); the
 // producer/MMA warpgroup needs few, the softmax and dQ-drain warpgroups more.
@@ -257,6 +260,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // arrives once its score loads are done and waits for the other before
   // storing.
   __shared__ __align__(8) uint64_t s_read, dp_read;
+  // The dQ drain stages a tile in shared memory before one bulk reduce-add.
+  __shared__ __align__(8) uint64_t dq_staged;
   __shared__ __align__(8) uint64_t qd_full[C::NST], qd_empty[C::NST], dq_full[C::NDQ], dq_free[C::NDQ];
   // Dynamic schedule: the producer claims work items from a global counter
   // and passes them to the other roles through this ring.
@@ -278,6 +283,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(&mma_drain, 1);
     mbar_init(&s_read, 256);
     mbar_init(&dp_read, 256);
+    mbar_init(&dq_staged, 128);
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(&qd_full[s], 1);
       mbar_init(&qd_empty[s], 1);
@@ -484,7 +490,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mma_ss(tmem + C::col_dq(b), smem_desc_sw128(aDS + s * 2048, C::CHUNK_BYTES, 1024),
                    smem_desc_sw128(aK + s * 2048, C::CHUNK_BYTES, 1024), IDESC_Q, s > 0 ? 1u : 0u);
           tc_commit(&dq_full[b]);
-          tc_commit(&qd_empty[st]);
+          if (!C::BULK_DQ) tc_commit(&qd_empty[st]);  // else the dQ drain returns it
           ++qd_iter;
           ++dq_iter;
           // dP^T of the next query tile (after the dQ drain when they share columns)
@@ -646,13 +652,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     regs_inc<136>();
     // ------------------------------------------------------------ dQ drain
-    // Read the whole dQ tile row out of tensor memory, hand the columns back
-    // to the MMA warp, then add the row into the fp32 accumulator.
+    // Read the whole dQ tile out of tensor memory and hand the columns back
+    // to the MMA warp, then add the tile into the fp32 accumulator (see
+    // Cfg::BULK_DQ).  With the bulk path the tile's Q/dO stage, dead by then
+    // (every product that reads it has completed), holds the tile in the
+    // accumulator's tiled layout for one bulk reduce-add, after which the
+    // stage goes back to the producer.
     const int quarter = warp & 3;
     const int qr = quarter * 32 + lane;
     const uint32_t lane_bits = uint32_t(quarter * 32) << 16;
+    const bool leader = warp == 12 && lane == 0;
     uint32_t dq_iter = 0;
-    bool ok = true;
+    bool ok = true, bulk_issued = false;
     for (uint32_t k = 0;; ++k) {
       int idx;
       ok = take_item_warp(k, idx);
@@ -660,6 +671,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const Item it = item_at(p, idx);
       for (int i = next_q(p, it.j, 0); i < p.nq; i = next_q(p, it.j, i + 1)) {
         const uint32_t b = dq_iter % C::NDQ;
+        const uint32_t st = dq_iter % C::NST;
         ok = mbar_wait_warp(&dq_full[b], (dq_iter / C::NDQ) & 1, w);
         if (!ok) break;
         tc_fence_after();
@@ -669,15 +681,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_wait_ld();
         tc_fence_before();
         mbar_arrive(&dq_free[b]);
-        // tiled accumulator: columns 4e..4e+3 of row qr at e * 512 + qr * 4
-        float* dst = p.dq_acc + ((size_t)it.bh * p.Npad + (size_t)i * BQ) * D + qr * 4;
+        if (C::BULK_DQ) {
+          // tiled layout: columns 4e..4e+3 of row qr at byte e * 2048 + qr * 16
+          uint8_t* stage = sQD + st * 2 * C::TILE_BYTES;
 #pragma unroll
-        for (int e = 0; e < D / 4; ++e)
-          red_add_v4(dst + e * 512, __uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                     __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+          for (int e = 0; e < D / 4; ++e)
+            *reinterpret_cast<uint4*>(stage + e * 2048 + qr * 16) =
+                make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+          fence_proxy_async_smem();
+          mbar_arrive(&dq_staged);
+          if (leader) {
+            ok = mbar_wait(&dq_staged, dq_iter & 1, w);
+            if (ok) {
+              bulk_reduce_add_f32(p.dq_acc + ((size_t)it.bh * p.Npad + (size_t)i * BQ) * D, stage, 128 * D * 4);
+              bulk_commit_group();
+              bulk_issued = true;
+              bulk_wait_read_all();
+              mbar_arrive(&qd_empty[st]);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+        } else {
+          // tiled accumulator: columns 4e..4e+3 of row qr at e * 512 + qr * 4;
+          // one warp instruction covers 512 contiguous bytes
+          float* dst = p.dq_acc + ((size_t)it.bh * p.Npad + (size_t)i * BQ) * D + qr * 4;
+#pragma unroll
+          for (int e = 0; e < D / 4; ++e)
+            red_add_v4(dst + e * 512, __uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                       __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        }
         ++dq_iter;
       }
     }
+    if (leader && bulk_issued) bulk_wait_all();
   }
 
   tc_fence_before();
