@@ -188,6 +188,14 @@ struct Cfg {
   // the stage that long would starve the producer, so each drain thread adds
   // its row with vector reductions and the MMA warp returns the stage.
   static constexpr bool BULK_DQ = D == 64;
+  // Registers per thread of the producer/MMA, softmax and drain warpgroups
+  // (setmaxnreg).  Launch: 512 threads x 128; 128 x (REG_CTL + 2 REG_SMX +
+  // REG_DRN) must stay <= 65536.  Chosen so that ptxas spills nothing (d=128)
+  // or next to nothing (d=64).
+  static constexpr uint32_t REG_CTL = D == 128 ? 104 : 88;
+  static constexpr uint32_t REG_SMX = 136;
+  static constexpr uint32_t REG_DRN = 136;
+  static_assert(REG_CTL + 2 * REG_SMX + REG_DRN <= 512, "register split exceeds the launch");
 };
 
 struct Params {
@@ -242,9 +250,6 @@ __device__ __forceinline__ int next_q(const Params& p, int j, int i) {
 }
 
 
-// Register budget: the launch gives 128 per thread (512 threads); the
-// producer/MMA warpgroup needs few, the softmax and dQ-drain warpgroups more.
-// 128 threads x (88 + 136 + 136 + 136) = 63488 <= 65536, the launch total.
 
 template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -338,7 +343,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   };
 
   if (warp < 4) {
-    regs_dec<88>();
+    regs_dec<C::REG_CTL>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -508,7 +513,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
   } else if (warp < 12) {
-    regs_inc<136>();
+    regs_inc<C::REG_SMX>();
     // ------------------------------------------------------------ softmax
     const int quarter = warp & 3;
     const int hf = (warp - 4) >> 2;        // query half: columns [64 hf, 64 hf + 64)
@@ -536,8 +541,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float* sD = sL + 128;
         const bool key_live = key < p.N;
         const bool diag = p.mask_kind == FA_MASK_CAUSAL && i == it.j;
-        // ---- P^T = exp2(S^T * scale * log2e - LSE_i * log2e)
-        float pr[64];
+        // element masks only on the causal diagonal and a ragged last key tile
+        const bool masked = diag || (it.j + 1) * BK > p.N;
+        // ---- P^T = exp2(S^T * scale * log2e - LSE_i * log2e), kept packed
+        // as bf16 pairs (the form the dV product reads) for the dS step too.
+        uint32_t pk[32];
         {
           uint32_t sr[64];
           FA_TMEM_LD_X32(tmem + lane_bits + C::COL_S + hf * 64, sr);
@@ -549,29 +557,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             const float4 lv = l4[u];
-            const float lvv[4] = {lv.x, lv.y, lv.z, lv.w};
+            float pv[4] = {ex2_approx(fmaf(__uint_as_float(sr[4 * u + 0]), sl2, -lv.x)),
+                           ex2_approx(fmaf(__uint_as_float(sr[4 * u + 1]), sl2, -lv.y)),
+                           ex2_approx(fmaf(__uint_as_float(sr[4 * u + 2]), sl2, -lv.z)),
+                           ex2_approx(fmaf(__uint_as_float(sr[4 * u + 3]), sl2, -lv.w))};
+            if (masked) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int col = u * 4 + e;
-              float pv = ex2_approx(fmaf(__uint_as_float(sr[col]), sl2, -lvv[e]));
-              if (!key_live || (diag && hf * 64 + col < kr)) pv = 0.0f;
-              pr[col] = pv;
+              for (int e = 0; e < 4; ++e)
+                if (!key_live || (diag && hf * 64 + 4 * u + e < kr)) pv[e] = 0.0f;
             }
+            pk[2 * u] = pack_bf16x2(pv[0], pv[1]);
+            pk[2 * u + 1] = pack_bf16x2(pv[2], pv[3]);
           }
         }
-        {
-          uint32_t pk[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
-          ok = mbar_wait_warp(&s_read, par, w);
-          if (!ok) break;
-          tc_fence_after();
-          FA_TMEM_ST_X32(tmem + lane_bits + C::COL_P + hf * 32, pk);
-        }
+        ok = mbar_wait_warp(&s_read, par, w);
+        if (!ok) break;
+        tc_fence_after();
+        FA_TMEM_ST_X32(tmem + lane_bits + C::COL_P + hf * 32, pk);
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full);
-        // ---- dS^T = P^T * (dP^T - D)
+        // ---- dS^T = P^T * (dP^T - D), with P as the bf16 values above
         ok = mbar_wait_warp(&dp_full, par, w);
         if (!ok) break;
         tc_fence_after();
@@ -589,11 +595,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const float4 dv = d4[u];
-            const int c = cc * 32 + u * 4;
-            const float g0 = pr[c + 0] * (__uint_as_float(dr[u * 4 + 0]) - dv.x);
-            const float g1 = pr[c + 1] * (__uint_as_float(dr[u * 4 + 1]) - dv.y);
-            const float g2 = pr[c + 2] * (__uint_as_float(dr[u * 4 + 2]) - dv.z);
-            const float g3 = pr[c + 3] * (__uint_as_float(dr[u * 4 + 3]) - dv.w);
+            const uint32_t w0 = pk[cc * 16 + 2 * u], w1 = pk[cc * 16 + 2 * u + 1];
+            const float g0 = __uint_as_float(w0 << 16) * (__uint_as_float(dr[u * 4 + 0]) - dv.x);
+            const float g1 = __uint_as_float(w0 & 0xffff0000u) * (__uint_as_float(dr[u * 4 + 1]) - dv.y);
+            const float g2 = __uint_as_float(w1 << 16) * (__uint_as_float(dr[u * 4 + 2]) - dv.z);
+            const float g3 = __uint_as_float(w1 & 0xffff0000u) * (__uint_as_float(dr[u * 4 + 3]) - dv.w);
             dk[cc * 16 + u * 2 + 0] = pack_bf16x2(g0, g1);
             dk[cc * 16 + u * 2 + 1] = pack_bf16x2(g2, g3);
           }
@@ -650,7 +656,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
     }
   } else {
-    regs_inc<136>();
+    regs_inc<C::REG_DRN>();
     // ------------------------------------------------------------ dQ drain
     // Read the whole dQ tile out of tensor memory and hand the columns back
     // to the MMA warp, then add the tile into the fp32 accumulator (see
