@@ -196,6 +196,9 @@ struct Cfg {
   static constexpr uint32_t REG_SMX = 136;
   static constexpr uint32_t REG_DRN = 136;
   static_assert(REG_CTL + 2 * REG_SMX + REG_DRN <= 512, "register split exceeds the launch");
+  // setmaxnreg.dec may only lower and setmaxnreg.inc only raise the 128
+  // registers a thread starts with (anything else is an illegal instruction).
+  static_assert(REG_CTL <= 128 && REG_SMX >= 128 && REG_DRN >= 128, "setmaxnreg direction");
 };
 
 struct Params {

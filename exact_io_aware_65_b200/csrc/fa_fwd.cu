@@ -158,8 +158,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // Registers: 384 threads x 168 at launch; the producer/MMA warpgroup gives
   // much of its share to the two softmax warpgroups: 128 x (88 + 208 + 208)
   // = 64512, the launch total.
+  static_assert(88 + 208 + 208 <= 3 * 168, "register split exceeds the launch");
   if (warp < 4) {
-    regs_dec<88>();
+    regs_dec<88>();  // may only lower the 168 registers of the launch
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -306,7 +307,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
   } else {
-    regs_inc<208>();
+    regs_inc<208>();  // may only raise them
     // ------------------------------------------------------------ softmax
     const int t = (warp - 4) >> 2;         // query tile of this warpgroup
     const int quarter = warp & 3;          // tensor-memory lane quarter
