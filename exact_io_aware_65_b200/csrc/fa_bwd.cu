@@ -182,19 +182,24 @@ struct Cfg {
   // buffers after dK.
   static constexpr int NDQ = D == 64 ? 2 : 1;
   __host__ __device__ static constexpr int col_dq(int b) { return D == 128 ? 128 : 384 + 64 * b; }
-  // How a dQ tile reaches the fp32 accumulator.  d = 64 (four Q/dO stages):
-  // staged in its own dead Q/dO stage and added with one bulk reduce-add,
-  // the stage then returned to the producer.  d = 128 (two stages): holding
-  // the stage that long would starve the producer, so each drain thread adds
-  // its row with vector reductions and the MMA warp returns the stage.
-  static constexpr bool BULK_DQ = D == 64;
+  // A dQ tile (fp32, 4 * 128 * D bytes) reaches the accumulator by bulk
+  // reduce-adds from shared memory.  d = 64: the tile's whole Q/dO stage
+  // (2 * TILE_BYTES, dead once dQ has been computed) holds it for one bulk
+  // add, after which the drain returns both halves of the stage.  d = 128:
+  // with two stages, holding the Q half that long would starve the producer,
+  // so only the dO half holds it, in two halves added one after the other,
+  // and the MMA warp returns the Q half right after the dQ product.
+  static constexpr int DQ_PARTS = D == 128 ? 2 : 1;
+  static constexpr int DQ_PART_BYTES = 4 * 128 * D / DQ_PARTS;
+  static constexpr int DQ_SLOT_OFF = D == 128 ? TILE_BYTES : 0;  // within the stage
+  static_assert(DQ_SLOT_OFF + DQ_PART_BYTES <= 2 * TILE_BYTES, "dQ part exceeds its stage");
   // Registers per thread of the producer/MMA, softmax and drain warpgroups
   // (setmaxnreg).  Launch: 512 threads x 128; 128 x (REG_CTL + 2 REG_SMX +
   // REG_DRN) must stay <= 65536.  Chosen so that ptxas spills nothing (d=128)
   // or next to nothing (d=64).
   static constexpr uint32_t REG_CTL = D == 128 ? 104 : 88;
-  static constexpr uint32_t REG_SMX = 136;
-  static constexpr uint32_t REG_DRN = 136;
+  static constexpr uint32_t REG_SMX = D == 128 ? 128 : 136;
+  static constexpr uint32_t REG_DRN = 152;
   static_assert(REG_CTL + 2 * REG_SMX + REG_DRN <= 512, "register split exceeds the launch");
   // setmaxnreg.dec may only lower and setmaxnreg.inc only raise the 128
   // registers a thread starts with (anything else is an illegal instruction).
@@ -224,10 +229,6 @@ struct Item {
 // p.group, so the query-side tiles and dQ rows in flight at any time belong
 // to a few heads and stay in L2; within a group low key tiles come first
 // (under a causal mask they meet the most query tiles and run longest).
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
 
 __device__ __forceinline__ Item item_at(const Params& p, int idx) {
   const int per_group = p.group * p.nq;
@@ -268,9 +269,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // arrives once its score loads are done and waits for the other before
   // storing.
   __shared__ __align__(8) uint64_t s_read, dp_read;
-  // The dQ drain stages a tile in shared memory before one bulk reduce-add.
-  __shared__ __align__(8) uint64_t dq_staged;
-  __shared__ __align__(8) uint64_t qd_full[C::NST], qd_empty[C::NST], dq_full[C::NDQ], dq_free[C::NDQ];
+  // The dQ drain stages a tile in shared memory, in one or two parts, before
+  // each bulk reduce-add (dq_staged[h]: all 128 drain threads have written
+  // part h; dq_half: the first part has been read out).  One barrier per
+  // part, each completing one phase per tile.
+  __shared__ __align__(8) uint64_t dq_staged[2], dq_half;
+  // Each stage holds a query tile's Q (with its LSE values) and dO (with its
+  // D values), filled and released independently: the dQ drain releases
+  // what held the tile's dQ for its bulk reduction, the MMA warp the Q half
+  // when that was not needed (Cfg::DQ_PARTS).
+  __shared__ __align__(8) uint64_t q_full[C::NST], q_empty[C::NST], do_full[C::NST], do_empty[C::NST];
+  __shared__ __align__(8) uint64_t dq_full[C::NDQ], dq_free[C::NDQ];
   // Dynamic schedule: the producer claims work items from a global counter
   // and passes them to the other roles through this ring.
   __shared__ __align__(8) uint64_t item_full[RING], item_empty[RING];
@@ -291,10 +300,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(&mma_drain, 1);
     mbar_init(&s_read, 256);
     mbar_init(&dp_read, 256);
-    mbar_init(&dq_staged, 128);
+    mbar_init(&dq_staged[0], 128);
+    mbar_init(&dq_staged[1], 128);
+    mbar_init(&dq_half, 1);
     for (int s = 0; s < C::NST; ++s) {
-      mbar_init(&qd_full[s], 1);
-      mbar_init(&qd_empty[s], 1);
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+      mbar_init(&do_full[s], 1);
+      mbar_init(&do_empty[s], 1);
     }
     for (int b = 0; b < C::NDQ; ++b) {
       mbar_init(&dq_full[b], 1);
@@ -351,7 +364,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t item_iter = 0, qd_iter = 0;
-      bool ok = true;
+      bool ok = true, q_only = false;  // q_only: the last tile's dO load was never issued
       for (;; ++item_iter) {
         const uint32_t slot = item_iter % RING;
         ok = mbar_wait(&item_empty[slot], ((item_iter / RING) & 1) ^ 1, w);
@@ -372,28 +385,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         for (int i = next_q(p, it.j, 0); i < p.nq; i = next_q(p, it.j, i + 1)) {
           const uint32_t st = qd_iter % C::NST;
-          ok = mbar_wait(&qd_empty[st], ((qd_iter / C::NST) & 1) ^ 1, w);
-          if (!ok) break;
-          mbar_arrive_expect_tx(&qd_full[st], 2 * C::TILE_BYTES + 1024);
+          const uint32_t par = ((qd_iter / C::NST) & 1) ^ 1;
           uint8_t* q = sQD + st * 2 * C::TILE_BYTES;
-#pragma unroll
-          for (int c = 0; c < C::CHUNKS; ++c) {
-            tma_load_3d(q + c * C::CHUNK_BYTES, &mapQ, &qd_full[st], c * 64, i * BQ, it.bh);
-            tma_load_3d(q + C::TILE_BYTES + c * C::CHUNK_BYTES, &mapdO, &qd_full[st], c * 64, i * BQ, it.bh);
-          }
           const size_t row0 = (size_t)it.bh * p.Npad + (size_t)i * BQ;
           uint8_t* ld = smem + C::OFF_LD + st * 1024;
-          bulk_load(ld, p.L2w + row0, 512, &qd_full[st]);
-          bulk_load(ld + 512, p.Dw + row0, 512, &qd_full[st]);
+          ok = mbar_wait(&q_empty[st], par, w);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&q_full[st], C::TILE_BYTES + 512);
+#pragma unroll
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_3d(q + c * C::CHUNK_BYTES, &mapQ, &q_full[st], c * 64, i * BQ, it.bh);
+          bulk_load(ld, p.L2w + row0, 512, &q_full[st]);
+          ok = mbar_wait(&do_empty[st], par, w);
+          if (!ok) {
+            ++qd_iter;
+            q_only = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&do_full[st], C::TILE_BYTES + 512);
+#pragma unroll
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_3d(q + C::TILE_BYTES + c * C::CHUNK_BYTES, &mapdO, &do_full[st], c * 64, i * BQ, it.bh);
+          bulk_load(ld + 512, p.Dw + row0, 512, &do_full[st]);
           ++qd_iter;
         }
+        if (!ok) break;
       }
       if (!ok) {
         const uint64_t dl = globaltimer_ns() + 100000000ull;
         const uint32_t n = qd_iter < (uint32_t)C::NST ? qd_iter : (uint32_t)C::NST;
         for (uint32_t k = 0; k < n; ++k) {
           const uint32_t q = qd_iter - 1 - k;
-          mbar_drain_wait(&qd_full[q % C::NST], (q / C::NST) & 1, dl);
+          mbar_drain_wait(&q_full[q % C::NST], (q / C::NST) & 1, dl);
+          if (!(k == 0 && q_only)) mbar_drain_wait(&do_full[q % C::NST], (q / C::NST) & 1, dl);
         }
         if (item_iter > 0) mbar_drain_wait(&kv_full, (item_iter - 1) & 1, dl);
       }
@@ -421,11 +445,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       // dP^T = V dO^T.  With d = 128 the dP^T columns hold the previous dQ
       // tile until the drain warps have read it.
-      auto issue_dp = [&](uint32_t st) -> bool {
+      auto issue_dp = [&](uint32_t tile) -> bool {
+        const uint32_t st = tile % C::NST;
+        if (!mbar_wait(&do_full[st], (tile / C::NST) & 1, w)) return false;
         if (D == 128 && dq_iter > 0) {
           if (!mbar_wait(&dq_free[0], (dq_iter - 1) & 1, w)) return false;
-          tc_fence_after();
         }
+        tc_fence_after();
         const uint32_t adO = aQD + st * 2 * C::TILE_BYTES + C::TILE_BYTES;
 #pragma unroll
         for (int s = 0; s < D / 16; ++s) {
@@ -446,12 +472,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!ok) break;
         int i = next_q(p, it.j, 0);
         if (i < p.nq) {
-          ok = mbar_wait(&qd_full[qd_iter % C::NST], (qd_iter / C::NST) & 1, w);
+          ok = mbar_wait(&q_full[qd_iter % C::NST], (qd_iter / C::NST) & 1, w);
           if (!ok) break;
           tc_fence_after();
           issue_s(qd_iter % C::NST);
           issued = true;
-          ok = issue_dp(qd_iter % C::NST);
+          ok = issue_dp(qd_iter);
           if (!ok) break;
         }
         for (int n = 0; ok && i < p.nq; ++n) {
@@ -473,7 +499,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // by the dV product just issued, and its softmax can then overlap
           // the dK, dQ and next dP products.
           if (inext < p.nq) {
-            ok = mbar_wait(&qd_full[stn], ((qd_iter + 1) / C::NST) & 1, w);
+            ok = mbar_wait(&q_full[stn], ((qd_iter + 1) / C::NST) & 1, w);
             if (!ok) break;
             tc_fence_after();
             issue_s(stn);
@@ -498,11 +524,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mma_ss(tmem + C::col_dq(b), smem_desc_sw128(aDS + s * 2048, C::CHUNK_BYTES, 1024),
                    smem_desc_sw128(aK + s * 2048, C::CHUNK_BYTES, 1024), IDESC_Q, s > 0 ? 1u : 0u);
           tc_commit(&dq_full[b]);
-          if (!C::BULK_DQ) tc_commit(&qd_empty[st]);  // else the dQ drain returns it
+          if (C::DQ_PARTS == 2) tc_commit(&q_empty[st]);  // the rest goes back via the dQ drain
           ++qd_iter;
           ++dq_iter;
           // dP^T of the next query tile (after the dQ drain when they share columns)
-          if (inext < p.nq) ok = issue_dp(stn);
+          if (inext < p.nq) ok = issue_dp(qd_iter);
           i = inext;
         }
         if (!ok) break;
@@ -661,12 +687,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     regs_inc<C::REG_DRN>();
     // ------------------------------------------------------------ dQ drain
-    // Read the whole dQ tile out of tensor memory and hand the columns back
-    // to the MMA warp, then add the tile into the fp32 accumulator (see
-    // Cfg::BULK_DQ).  With the bulk path the tile's Q/dO stage, dead by then
-    // (every product that reads it has completed), holds the tile in the
-    // accumulator's tiled layout for one bulk reduce-add, after which the
-    // stage goes back to the producer.
+    // Read the whole dQ tile out of tensor memory, hand the columns back to
+    // the MMA warp, then add the tile into the fp32 accumulator with bulk
+    // reduce-adds (the TMA engine: vector reductions from the threads
+    // saturated the load/store pipe that everything else here also uses).
     const int quarter = warp & 3;
     const int qr = quarter * 32 + lane;
     const uint32_t lane_bits = uint32_t(quarter * 32) << 16;
@@ -690,36 +714,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_wait_ld();
         tc_fence_before();
         mbar_arrive(&dq_free[b]);
-        if (C::BULK_DQ) {
-          // tiled layout: columns 4e..4e+3 of row qr at byte e * 2048 + qr * 16
-          uint8_t* stage = sQD + st * 2 * C::TILE_BYTES;
+        // Stage the tile in its dead stage (the products that read it have
+        // completed) in the accumulator's tiled layout, columns 4e..4e+3 of
+        // row qr at byte e * 2048 + qr * 16 of a part, and add each part with
+        // one bulk reduce-add (Cfg::DQ_PARTS).
+        constexpr int GROUPS = D / 4 / C::DQ_PARTS;  // 4-column groups per part
+        uint8_t* slot = sQD + st * 2 * C::TILE_BYTES + C::DQ_SLOT_OFF;
+        float* dst = p.dq_acc + ((size_t)it.bh * p.Npad + (size_t)i * BQ) * D;
 #pragma unroll
-          for (int e = 0; e < D / 4; ++e)
-            *reinterpret_cast<uint4*>(stage + e * 2048 + qr * 16) =
-                make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+        for (int h = 0; h < C::DQ_PARTS; ++h) {
+          if (h == 1) {
+            ok = mbar_wait_warp(&dq_half, dq_iter & 1, w);  // first part read out
+            if (!ok) break;
+          }
+#pragma unroll
+          for (int e = 0; e < GROUPS; ++e) {
+            const int g = h * GROUPS + e;
+            *reinterpret_cast<uint4*>(slot + e * 2048 + qr * 16) =
+                make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+          }
           fence_proxy_async_smem();
-          mbar_arrive(&dq_staged);
+          // A warp that has run ahead arrives only once the previous tile's
+          // phase of this barrier is complete (else its arrival would count
+          // toward that phase).
+          if (dq_iter > 0) {
+            ok = mbar_wait_warp(&dq_staged[h], (dq_iter - 1) & 1, w);
+            if (!ok) break;
+          }
+          mbar_arrive(&dq_staged[h]);
           if (leader) {
-            ok = mbar_wait(&dq_staged, dq_iter & 1, w);
+            ok = mbar_wait(&dq_staged[h], dq_iter & 1, w);
             if (ok) {
-              bulk_reduce_add_f32(p.dq_acc + ((size_t)it.bh * p.Npad + (size_t)i * BQ) * D, stage, 128 * D * 4);
+              bulk_reduce_add_f32(dst + h * GROUPS * 512, slot, C::DQ_PART_BYTES);
               bulk_commit_group();
               bulk_issued = true;
               bulk_wait_read_all();
-              mbar_arrive(&qd_empty[st]);
+              if (h + 1 < C::DQ_PARTS) {
+                mbar_arrive(&dq_half);
+              } else {
+                if (C::DQ_PARTS == 1) mbar_arrive(&q_empty[st]);
+                mbar_arrive(&do_empty[st]);
+              }
             }
           }
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
           if (!ok) break;
-        } else {
-          // tiled accumulator: columns 4e..4e+3 of row qr at e * 512 + qr * 4;
-          // one warp instruction covers 512 contiguous bytes
-          float* dst = p.dq_acc + ((size_t)it.bh * p.Npad + (size_t)i * BQ) * D + qr * 4;
-#pragma unroll
-          for (int e = 0; e < D / 4; ++e)
-            red_add_v4(dst + e * 512, __uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                       __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
         }
+        if (!ok) break;
         ++dq_iter;
       }
     }

@@ -102,3 +102,36 @@ def test_bwd_workloads_one_head(name):
     ref = oracle.bwd(sl(x["Q"]), sl(x["K"]), sl(x["V"]), sl(x["dO"]), w.mask, x["mask"], w.scale)
     for nm, g in (("dQ", dQ), ("dK", dK), ("dV", dV)):
         assert_grad(f64(sl(g)), ref[nm][0:1], nm, name)
+
+
+@pytest.mark.parametrize("name", workloads.ORDER)
+def test_bwd_workloads_every_head(name):
+    """Full-size workloads in the benchmark's launch configuration, checked
+    in every head: sampled dQ rows (first, last and tile-boundary rows among
+    them) against the oracle's per-row gradient, and dK, dV through the
+    identities sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i (rows of dS sum to
+    zero, rows of P to one; every query row of these workloads sees a key)."""
+    w = workloads.WORKLOADS[name]
+    x = workloads.make_inputs(w, 3)
+    dQ, dK, dV = run(w, x)
+    BH = w.B * w.H
+    rng = np.random.default_rng(11)
+    per = 6
+    rows = rng.integers(0, w.N, (BH, per))
+    rows[:, 0], rows[:, 1] = 0, w.N - 1
+    rows[:, 2], rows[:, 3] = min(127, w.N - 1), min(128, w.N - 1)
+    heads = np.repeat(np.arange(BH), per)
+    rows = rows.reshape(-1)
+    _, _, dQs = oracle.rows(x["Q"], x["K"], x["V"], heads, rows, dO=x["dO"], mask_kind=w.mask,
+                            block_mask=x["mask"], scale=w.scale)
+    g = f64(dQ).reshape(BH, w.N, w.d)[heads, rows].reshape(BH, per, w.d)
+    ref = dQs.reshape(BH, per, w.d)
+    for h in range(BH):
+        assert_grad(g[h], ref[h], "dQ", f"{name} head {h}")
+    dk = f64(dK).reshape(BH, w.N, w.d)
+    dv = f64(dV).reshape(BH, w.N, w.d)
+    do = f64(x["dO"]).reshape(BH, w.N, w.d)
+    kscale = np.abs(dk).sum(axis=1).max(axis=1)
+    assert (np.abs(dk.sum(axis=1)).max(axis=1) <= 2e-2 * kscale + 1e-6).all()
+    vscale = np.abs(do).sum(axis=1).max(axis=1)
+    assert (np.abs(dv.sum(axis=1) - do.sum(axis=1)).max(axis=1) <= 2e-2 * vscale).all()
