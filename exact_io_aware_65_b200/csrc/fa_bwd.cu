@@ -369,7 +369,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t slot = item_iter % RING;
         ok = mbar_wait(&item_empty[slot], ((item_iter / RING) & 1) ^ 1, w);
         if (!ok) break;
-        int idx = (int)atomicAdd(p.sched, 1u);
+        // CTA b starts on item b, then claims items gridDim.x, gridDim.x + 1, ...
+        int idx = item_iter == 0 ? (int)blockIdx.x : (int)gridDim.x + (int)atomicAdd(p.sched, 1u);
         if (idx > p.n_items) idx = p.n_items;
         item_ring[slot] = idx;
         mbar_arrive(&item_full[slot]);

@@ -10,8 +10,9 @@
 // B200 mapping (one persistent CTA per SM, 384 threads):
 //   warp 0        TMA producer: two 128-row Q tiles per work item, then a ring
 //                 of K and V tiles (128 keys x d, 128-byte swizzle).
-//   warp 1        MMA issuer (one thread): S_t = Q_t K_j^T into tensor memory
-//                 (fp32), and O_t += P_t V_j with P_t read from tensor memory.
+//   warps 1(, 2)  MMA issuer(s), one thread each (Cfg::ISSUERS): S_t = Q_t K_j^T
+//                 into tensor memory (fp32), and O_t += P_t V_j with P_t read
+//                 from tensor memory.
 //   warps 4..7    softmax for query tile 0; warps 8..11 for query tile 1.
 //                 Thread r owns query row r: it reads its score row from
 //                 tensor memory, keeps the row max m and row sum l in
@@ -30,6 +31,8 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <atomic>
+
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -39,6 +42,17 @@ namespace fwd {
 constexpr int BM = 128;              // query rows per tile
 constexpr int BN = 128;              // keys per tile
 constexpr int NUM_THREADS = 384;
+constexpr int RING = 4;              // depth of the item ring the producer fills
+
+// Dynamic schedule.  CTA b starts on item b; after that each CTA claims
+// items gridDim.x, gridDim.x + 1, ... from a counter.  Each launch takes one
+// of SCHED_SLOTS counters (in turn, on the host), and the last CTA to stop
+// claiming puts it back to zero.  Launches that run at the same time (other
+// streams) use other slots, so at most SCHED_SLOTS forward launches may be
+// in flight at once.
+constexpr uint32_t SCHED_SLOTS = 4096;
+__device__ uint32_t g_claim[SCHED_SLOTS];  // dynamic claims so far
+__device__ uint32_t g_done[SCHED_SLOTS];   // CTAs that stopped claiming
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 constexpr float LN2 = 0.69314718055994530942f;
 
@@ -49,6 +63,14 @@ struct Cfg {
   static constexpr int CHUNK_BYTES = BN * 128;   // one chunk of a tile
   static constexpr int NSLOT = D == 64 ? 8 : 4;  // K/V ring slots
   static constexpr int SMEM_BYTES = 2 * TILE_BYTES + NSLOT * TILE_BYTES + 1024;
+  // MMA issuer threads.  Issuing blocks while the tensor core's queue is
+  // full, so with one issuer a tile's PV can wait behind the other tile's
+  // products.  d = 64: one issuer per query tile (short products, so the
+  // decoupling wins).  d = 128: one issuer for both tiles, which keeps each
+  // tile's PV and next QK^T back to back on the tensor core (interleaving
+  // the two tiles' products delays both tiles' next scores).
+  static constexpr int ISSUERS = D == 64 ? 2 : 1;
+  static constexpr int CONSUMERS = ISSUERS + 8;  // of the item ring: issuers + softmax warps
 };
 
 struct Params {
@@ -60,6 +82,7 @@ struct Params {
   float* LSE;
   uint64_t timeout_ns;
   uint32_t* status;
+  uint32_t slot;  // scheduler counter slot of this launch
 };
 
 struct Item {
@@ -70,7 +93,8 @@ struct Item {
 // Work item idx -> (head, pair of query tiles).  Heads are taken in groups
 // of p.group so that the K/V tiles in flight belong to a few heads and stay
 // in L2; within a group later query tiles come first, so that under a causal
-// mask the longest items start earliest.
+// mask the longest items start earliest (and, claimed dynamically, the short
+// ones fill in at the end).
 __device__ __forceinline__ Item item_at(const Params& p, int idx) {
   Item it;
   const int per_group = p.group * p.n_pairs;
@@ -115,9 +139,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sQ = smem;                        // 2 tiles
   uint8_t* sKV = smem + 2 * C::TILE_BYTES;   // NSLOT tiles
 
-  __shared__ __align__(8) uint64_t q_full, q_empty, mma_drain;
+  __shared__ __align__(8) uint64_t q_full, q_empty, mma_drain[2];
   __shared__ __align__(8) uint64_t kv_full[C::NSLOT], kv_empty[C::NSLOT];
   __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_full[2];
+  // The producer claims work items and passes them to the other roles.
+  __shared__ __align__(8) uint64_t item_full[RING], item_empty[RING];
+  __shared__ int item_ring[RING];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -126,16 +153,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(&q_full, 1);
-    mbar_init(&q_empty, 1);
-    mbar_init(&mma_drain, 1);
+    mbar_init(&q_empty, C::ISSUERS);  // one commit from each MMA issuer
+    mbar_init(&mma_drain[0], 1);
+    mbar_init(&mma_drain[1], 1);
     for (int i = 0; i < C::NSLOT; ++i) {
       mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&kv_empty[i], C::ISSUERS);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], BM);
       mbar_init(&o_full[t], 1);
+    }
+    for (int r = 0; r < RING; ++r) {
+      mbar_init(&item_full[r], 1);
+      mbar_init(&item_empty[r], C::CONSUMERS);
     }
     fence_barrier_init();
   }
@@ -155,6 +187,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = tmem_base_sh;
   const WaitCtx w{p.timeout_ns, &abort_flag, p.status};
 
+  auto take_item = [&](uint32_t k, int& idx) -> bool {
+    const uint32_t slot = k % RING;
+    if (!mbar_wait(&item_full[slot], (k / RING) & 1, w)) return false;
+    idx = *reinterpret_cast<volatile int*>(&item_ring[slot]);
+    mbar_arrive(&item_empty[slot]);
+    return true;
+  };
+  auto take_item_warp = [&](uint32_t k, int& idx) -> bool {
+    const uint32_t slot = k % RING;
+    if (!mbar_wait_warp(&item_full[slot], (k / RING) & 1, w)) return false;
+    idx = *reinterpret_cast<volatile int*>(&item_ring[slot]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&item_empty[slot]);
+    return true;
+  };
+
   // Registers: 384 threads x 168 at launch; the producer/MMA warpgroup gives
   // much of its share to the two softmax warpgroups: 128 x (88 + 208 + 208)
   // = 64512, the launch total.
@@ -166,7 +214,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       uint32_t kv_iter = 0, item_iter = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_iter) {
+      for (;; ++item_iter) {
+        const uint32_t slot = item_iter % RING;
+        ok = mbar_wait(&item_empty[slot], ((item_iter / RING) & 1) ^ 1, w);
+        if (!ok) break;
+        int idx = item_iter == 0 ? (int)blockIdx.x : (int)gridDim.x + (int)atomicAdd(&g_claim[p.slot], 1u);
+        if (idx > p.n_items) idx = p.n_items;
+        item_ring[slot] = idx;
+        mbar_arrive(&item_full[slot]);
+        if (idx >= p.n_items) break;
         const Item it = item_at(p, idx);
         ok = mbar_wait(&q_empty, (item_iter & 1) ^ 1, w);
         if (!ok) break;
@@ -194,6 +250,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ++kv_iter;
           }
         }
+        if (!ok) break;
+      }
+      // This CTA claims no more (its last claim ran past the end, or it
+      // aborted); the last CTA to get here resets the counter slot.
+      if (atomicAdd(&g_done[p.slot], 1u) == gridDim.x - 1) {
+        g_claim[p.slot] = 0u;
+        g_done[p.slot] = 0u;
       }
       if (!ok) {
         // Let the loads already issued land before the CTA's shared memory
@@ -207,9 +270,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (item_iter > 0) mbar_drain_wait(&q_full, (item_iter - 1) & 1, dl);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || (C::ISSUERS == 2 && warp == 2)) {
+    // ------------------------------------------------------------ MMA issuers
+    // Cfg::ISSUERS threads; issuer u handles query tiles [t_lo, t_hi).  Each
+    // walks every key step of every item and commits every K/V slot and the
+    // Q tiles once (those barriers count one arrival per issuer).  Per key
+    // step and tile: O_t += P_t V_j, then S_t = Q_t K_{j+1}^T into the same
+    // columns (after the PV that reads P_t, in issue order).
     if (lane == 0) {
+      const int t_lo = C::ISSUERS == 2 ? warp - 1 : 0;
+      const int t_hi = C::ISSUERS == 2 ? warp : 2;
       constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(BM, D, 0, 1);
       const uint32_t sQ_addr = smem_u32(sQ);
@@ -226,6 +296,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mma_ss(tmem + t * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), IDESC_S,
                  s > 0 ? 1u : 0u);
         }
+        tc_commit(&s_full[t]);
+        issued = true;
       };
       auto issue_pv = [&](int t, uint32_t vslot, uint32_t acc) {
         const uint32_t va = sKV_addr + vslot * C::TILE_BYTES;
@@ -236,39 +308,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       };
 
-      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++item_iter) {
+      for (;; ++item_iter) {
+        int idx;
+        ok = take_item(item_iter, idx);
+        if (!ok || idx >= p.n_items) break;
         const Item it = item_at(p, idx);
+        const int tiles = it.has1 ? 2 : 1;  // tiles [0, tiles) exist
         ok = mbar_wait(&q_full, item_iter & 1, w);
         if (!ok) break;
         tc_fence_after();
         const int e = kv_end(p, it);
         int j = next_union(p, it, 0);
+        int jn = j < e ? next_union(p, it, j + 1) : e;  // the key tile after j
         bool first_pv[2] = {true, true};
+        // Q is read only by the QK^T products: it goes back to the producer
+        // once the item's last one has been issued, so the next item's Q
+        // loads while this item's last softmax, PV and epilogue run.
+        bool q_released = false;
         if (j < e) {
           const uint32_t ks = kv_iter % C::NSLOT;
           ok = mbar_wait(&kv_full[ks], (kv_iter / C::NSLOT) & 1, w);
           if (!ok) break;
           tc_fence_after();
-          for (int t = 0; t < 2; ++t) {
-            if (t == 1 && !it.has1) continue;
-            if (!member(p, t == 0 ? it.q0 : it.q1, j)) continue;
-            issue_s(t, ks);
-            tc_commit(&s_full[t]);
-            issued = true;
-          }
+          for (int t = t_lo; t < t_hi && t < tiles; ++t)
+            if (member(p, t == 0 ? it.q0 : it.q1, j)) issue_s(t, ks);
           tc_commit(&kv_empty[ks]);
           ++kv_iter;
+          if (jn >= e) {
+            tc_commit(&q_empty);
+            q_released = true;
+          }
         }
         while (ok && j < e) {
-          const int jn = next_union(p, it, j + 1);
+          const int jnn = jn < e ? next_union(p, it, jn + 1) : e;
           const uint32_t vs = kv_iter % C::NSLOT;
           const uint32_t ksn = (kv_iter + 1) % C::NSLOT;
           ok = mbar_wait(&kv_full[vs], (kv_iter / C::NSLOT) & 1, w);
           if (ok && jn < e) ok = mbar_wait(&kv_full[ksn], ((kv_iter + 1) / C::NSLOT) & 1, w);
           if (!ok) break;
           tc_fence_after();
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (t == 1 && !it.has1) continue;
+          for (int t = t_lo; t < t_hi && t < tiles && ok; ++t) {
             const int qt = t == 0 ? it.q0 : it.q1;
             if (member(p, qt, j)) {
               ok = mbar_wait(&p_full[t], p_cnt[t] & 1, w);
@@ -278,31 +357,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               issue_pv(t, vs, first_pv[t] ? 0u : 1u);
               first_pv[t] = false;
             }
-            if (jn < e && member(p, qt, jn)) {
-              issue_s(t, ksn);
-              tc_commit(&s_full[t]);
-            }
+            if (jn < e && member(p, qt, jn)) issue_s(t, ksn);
           }
           if (!ok) break;
           tc_commit(&kv_empty[vs]);
           if (jn < e) {
             tc_commit(&kv_empty[ksn]);
             kv_iter += 2;
+            if (!q_released && jnn >= e) {
+              tc_commit(&q_empty);
+              q_released = true;
+            }
           } else {
             kv_iter += 1;
           }
           j = jn;
+          jn = jnn;
         }
         if (!ok) break;
-        tc_commit(&o_full[0]);
-        if (it.has1) tc_commit(&o_full[1]);
-        tc_commit(&q_empty);
+        for (int t = t_lo; t < t_hi && t < tiles; ++t) tc_commit(&o_full[t]);
+        if (!q_released) tc_commit(&q_empty);
       }
       if (issued) {
         // Every MMA issued by this thread must be finished before tensor
         // memory is released.
-        tc_commit(&mma_drain);
-        mbar_drain_wait(&mma_drain, 0, globaltimer_ns() + 100000000ull);
+        const int u = C::ISSUERS == 2 ? warp - 1 : 0;
+        tc_commit(&mma_drain[u]);
+        mbar_drain_wait(&mma_drain[u], 0, globaltimer_ns() + 100000000ull);
       }
     }
   }
@@ -319,7 +400,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
 
-    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x) {
+    for (uint32_t k = 0;; ++k) {
+      int idx;
+      ok = take_item_warp(k, idx);
+      if (!ok || idx >= p.n_items) break;
       const Item it = item_at(p, idx);
       if (t == 1 && !it.has1) continue;
       const int qt = t == 0 ? it.q0 : it.q1;
@@ -465,6 +549,8 @@ fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void
   p.LSE = LSE;
   p.timeout_ns = wait_timeout_ns();
   p.status = st;
+  static std::atomic<uint32_t> next_slot{0};
+  p.slot = next_slot.fetch_add(1u, std::memory_order_relaxed) % fwd::SCHED_SLOTS;
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (pr.d == 64) {
     constexpr int smem = fwd::Cfg<64>::SMEM_BYTES;
