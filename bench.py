@@ -22,6 +22,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -126,22 +127,33 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside)}
 
 
-def cpu_sample(w, x, mask, seed_rows=None):
-    """Time the fp64 oracle (fwd + bwd) on one head of the workload,
-    truncated to its first `n` positions; returns (TFLOP/s, seconds, desc)."""
-    import oracle  # test infrastructure: only the CPU-baseline leg uses it
+def cpu_sample(w, x, mask, seed_rows=None, heads=1):
+    """Time the fp64 oracle (fwd + bwd) on the first `heads` heads of the
+    workload, truncated to their first `seed_rows` positions; returns
+    (TFLOP/s, seconds, desc, threads)."""
+    import oracle  # test infrastructure: only the CPU-baseline legs use it
 
     n = seed_rows or w.N
-    sl = lambda t: t.reshape(w.B * w.H, w.N, w.d)[:1, :n].contiguous()
-    sub = w.with_(B=1, H=1, N=n)
+    sl = lambda t: t.reshape(w.B * w.H, w.N, w.d)[:heads, :n].contiguous()
+    sub = w.with_(B=1, H=heads, N=n)
     m = mask[: sub.nb, : sub.nb].contiguous() if mask is not None else None
     t0 = time.perf_counter()
     oracle.bwd(sl(x["Q"]), sl(x["K"]), sl(x["V"]), sl(x["dO"]), w.mask, m, w.scale)
     dt = time.perf_counter() - t0
     f = flops(sub, m)
-    desc = (f"fp64 oracle fwd+bwd (plain definition, all masked entries skipped) on head 0 of "
-            f"{w.name}, first {n} of {w.N} positions ({f['E']} kept score entries)")
+    desc = (f"fp64 oracle fwd+bwd (plain definition, all masked entries skipped) on heads 0..{heads - 1} of "
+            f"{w.name}, first {n} of {w.N} positions ({f['E']} kept score entries per head)")
     return (f["fwd"] + f["bwd"]) / dt / 1e12, dt, desc, oracle.num_threads()
+
+
+def cpu_baseline(w, x, mask, target_s=10.0):
+    """The oracle on a bounded sample of the workload: one head to gauge the
+    rate, then as many whole heads as take about `target_s` seconds."""
+    v, dt, desc, cores = cpu_sample(w, x, mask)
+    heads = max(1, min(w.B * w.H, int(math.ceil(target_s / max(dt, 1e-6)))))
+    if heads > 1:
+        v, dt, desc, cores = cpu_sample(w, x, mask, heads=heads)
+    return v, dt, desc, cores
 
 
 def reference_arm(args, w):
@@ -334,7 +346,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, dt, desc, cores = cpu_sample(w, x, mask_cpu)
+        v, dt, desc, cores = cpu_baseline(w, x, mask_cpu)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc, "seconds": dt}
 
     in_bytes = sum(t.numel() * t.element_size() for t in (Q, K, V, dO, O, LSE, dQ, dK, dV)) + ws.numel()
