@@ -42,7 +42,15 @@ def load(path: str):
     L.oracle_rows.argtypes = [_dp, _dp, _dp, _dp, i, i, i, i, _u8p, i, d,
                               _ip, _ip, i, _dp, _dp, _dp]
     L.oracle_probs.argtypes = [_dp, _dp, i, i, i, i, _u8p, i, d, _dp]
-    for f in (L.oracle_fwd, L.oracle_bwd, L.oracle_rows, L.oracle_probs):
+    # the same four with separate query and key counts (Nq, Nk)
+    L.oracle_fwd_qk.argtypes = [_dp, _dp, _dp, i, i, i, i, i, _u8p, i, d, _dp, _dp]
+    L.oracle_bwd_qk.argtypes = [_dp, _dp, _dp, _dp, i, i, i, i, i, _u8p, i, d,
+                                _dp, _dp, _dp, _dp, _dp, _dp]
+    L.oracle_rows_qk.argtypes = [_dp, _dp, _dp, _dp, i, i, i, i, i, _u8p, i, d,
+                                 _ip, _ip, i, _dp, _dp, _dp]
+    L.oracle_probs_qk.argtypes = [_dp, _dp, i, i, i, i, i, _u8p, i, d, _dp]
+    for f in (L.oracle_fwd, L.oracle_bwd, L.oracle_rows, L.oracle_probs,
+              L.oracle_fwd_qk, L.oracle_bwd_qk, L.oracle_rows_qk, L.oracle_probs_qk):
         f.restype = i
     return L
 
@@ -111,32 +119,42 @@ def _check(rc):
         raise RuntimeError(f"oracle call failed with code {rc}")
 
 
+def _nk(K, BH, d):
+    _, bh, Nk, dk = _shape(K)
+    if bh != BH or dk != d:
+        raise ValueError("K must have the same heads and head dimension as Q")
+    return Nk
+
+
 def fwd(Q, K, V, mask_kind="none", block_mask=None, scale=None, block=128):
-    """O [..., N, d] and LSE [..., N] in fp64."""
+    """O [..., Nq, d] and LSE [..., Nq] in fp64 (K, V [..., Nk, d])."""
     q, k, v = _f64(Q), _f64(K), _f64(V)
     lead, BH, N, d = _shape(q)
+    Nk = _nk(k, BH, d)
     scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
     kind, m, mp = _mask_args(block_mask, mask_kind)
     O = np.empty((BH, N, d))
     L = np.empty((BH, N))
-    _check(lib().oracle_fwd(_ptr(q), _ptr(k), _ptr(v), BH, N, d, kind, mp, block, scale,
-                            _ptr(O), _ptr(L)))
+    _check(lib().oracle_fwd_qk(_ptr(q), _ptr(k), _ptr(v), BH, N, Nk, d, kind, mp, block, scale,
+                               _ptr(O), _ptr(L)))
     return O.reshape(*lead, N, d), L.reshape(*lead, N)
 
 
 def bwd(Q, K, V, dO, mask_kind="none", block_mask=None, scale=None, block=128):
-    """dict with dQ, dK, dV [..., N, d] and O, LSE, D (fp64), all recomputed."""
+    """dict with dQ, O [..., Nq, d], dK, dV [..., Nk, d] and LSE, D [..., Nq]
+    (fp64), all recomputed."""
     q, k, v, do = _f64(Q), _f64(K), _f64(V), _f64(dO)
     lead, BH, N, d = _shape(q)
+    Nk = _nk(k, BH, d)
     scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
     kind, m, mp = _mask_args(block_mask, mask_kind)
-    out = {n: np.empty((BH, N, d)) for n in ("dQ", "dK", "dV", "O")}
+    out = {n: np.empty((BH, N if n in ("dQ", "O") else Nk, d)) for n in ("dQ", "dK", "dV", "O")}
     L = np.empty((BH, N))
     D = np.empty((BH, N))
-    _check(lib().oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), BH, N, d, kind, mp, block,
-                            scale, _ptr(out["dQ"]), _ptr(out["dK"]), _ptr(out["dV"]),
-                            _ptr(out["O"]), _ptr(L), _ptr(D)))
-    res = {n: a.reshape(*lead, N, d) for n, a in out.items()}
+    _check(lib().oracle_bwd_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(do), BH, N, Nk, d, kind, mp, block,
+                               scale, _ptr(out["dQ"]), _ptr(out["dK"]), _ptr(out["dV"]),
+                               _ptr(out["O"]), _ptr(L), _ptr(D)))
+    res = {n: a.reshape(*lead, a.shape[1], d) for n, a in out.items()}
     res["LSE"] = L.reshape(*lead, N)
     res["D"] = D.reshape(*lead, N)
     return res
@@ -149,6 +167,7 @@ def rows(Q, K, V, heads, rws, dO=None, mask_kind="none", block_mask=None, scale=
     q, k, v = _f64(Q), _f64(K), _f64(V)
     do = _f64(dO) if dO is not None else None
     lead, BH, N, d = _shape(q)
+    Nk = _nk(k, BH, d)
     scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
     kind, m, mp = _mask_args(block_mask, mask_kind)
     hs = np.ascontiguousarray(np.asarray(heads, dtype=np.int32))
@@ -157,18 +176,19 @@ def rows(Q, K, V, heads, rws, dO=None, mask_kind="none", block_mask=None, scale=
     O = np.empty((R, d))
     L = np.empty((R,))
     dQ = np.empty((R, d)) if do is not None else None
-    _check(lib().oracle_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(do), BH, N, d, kind, mp, block,
-                             scale, hs.ctypes.data_as(_ip), rs.ctypes.data_as(_ip), R,
-                             _ptr(O), _ptr(L), _ptr(dQ)))
+    _check(lib().oracle_rows_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(do), BH, N, Nk, d, kind, mp, block,
+                                scale, hs.ctypes.data_as(_ip), rs.ctypes.data_as(_ip), R,
+                                _ptr(O), _ptr(L), _ptr(dQ)))
     return (O, L, dQ) if do is not None else (O, L)
 
 
 def probs(Q, K, mask_kind="none", block_mask=None, scale=None, block=128):
-    """Softmax probabilities P [..., N, N] (small N only)."""
+    """Softmax probabilities P [..., Nq, Nk] (small sizes only)."""
     q, k = _f64(Q), _f64(K)
     lead, BH, N, d = _shape(q)
+    Nk = _nk(k, BH, d)
     scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
     kind, m, mp = _mask_args(block_mask, mask_kind)
-    P = np.empty((BH, N, N))
-    _check(lib().oracle_probs(_ptr(q), _ptr(k), BH, N, d, kind, mp, block, scale, _ptr(P)))
-    return P.reshape(*lead, N, N)
+    P = np.empty((BH, N, Nk))
+    _check(lib().oracle_probs_qk(_ptr(q), _ptr(k), BH, N, Nk, d, kind, mp, block, scale, _ptr(P)))
+    return P.reshape(*lead, N, Nk)

@@ -14,11 +14,16 @@ import test_oracle_pins as pins
 
 # (name, text in oracle.c, replacement, number of occurrences to replace)
 MUTANTS = [
-    ("causal_off_by_one", "case OR_MASK_CAUSAL: return j <= i;", "case OR_MASK_CAUSAL: return j < i;"),
-    ("block_mask_transposed", "s->bm[(size_t)(i / s->block) * s->nb + (j / s->block)]",
-     "s->bm[(size_t)(j / s->block) * s->nb + (i / s->block)]"),
+    ("causal_off_by_one", "case OR_MASK_CAUSAL: return j <= i + (s->Nk - s->Nq);",
+     "case OR_MASK_CAUSAL: return j < i + (s->Nk - s->Nq);"),
+    ("causal_offset_dropped", "case OR_MASK_CAUSAL: return j <= i + (s->Nk - s->Nq);",
+     "case OR_MASK_CAUSAL: return j <= i;"),
+    ("causal_offset_sign", "case OR_MASK_CAUSAL: return j <= i + (s->Nk - s->Nq);",
+     "case OR_MASK_CAUSAL: return j <= i + (s->Nq - s->Nk);"),
+    ("block_mask_transposed", "s->bm[(size_t)(i / s->block) * s->nbk + (j / s->block)]",
+     "s->bm[(size_t)(j / s->block) * s->nbk + (i / s->block)]"),
     ("lse_drops_max", "return m + log(l);", "return log(l);"),
-    ("no_normalisation", "for (int j = 0; j < s->N; ++j) S[j] /= l;", ""),
+    ("no_normalisation", "for (int j = 0; j < s->Nk; ++j) S[j] /= l;", ""),
     ("scale_dropped_in_scores", "S[j] = s->scale * dot(q, Kh + (size_t)j * s->d, s->d);",
      "S[j] = dot(q, Kh + (size_t)j * s->d, s->d);"),
     ("dS_sign", "double ds = P[j] * (dP[j] - Di);", "double ds = P[j] * (dP[j] + Di);"),
@@ -26,9 +31,9 @@ MUTANTS = [
      "\n                if (O)"),
     ("dK_transposed_operand", "dk[k] += ds * qi[k];", "dk[k] += ds * kj[k];"),
     ("dV_uses_dS", "dv[k] += p * doi[k];", "dv[k] += ds * doi[k];"),
-    ("D_dropped_in_pass2", "double ds = p * (dp - Dv[(size_t)h * N + i]);", "double ds = p * dp;"),
-    ("pv_wrong_row", "const double *v = V + hoff + (size_t)j * d;\n                    for (int k = 0; k < d; ++k) o[k] += P[j] * v[k];\n                }\n            }\n        free(P);\n    }\n    return err;\n}\n\n/* Backward",
-     "const double *v = V + hoff + (size_t)(N - 1 - j) * d;\n                    for (int k = 0; k < d; ++k) o[k] += P[j] * v[k];\n                }\n            }\n        free(P);\n    }\n    return err;\n}\n\n/* Backward"),
+    ("D_dropped_in_pass2", "double ds = p * (dp - Dv[(size_t)h * Nq + i]);", "double ds = p * dp;"),
+    ("pv_wrong_row", "const double *v = V + hk + (size_t)j * d;\n                    for (int k = 0; k < d; ++k) o[k] += P[j] * v[k];\n                }\n            }\n        free(P);\n    }\n    return err;\n}\n\nint oracle_fwd(",
+     "const double *v = V + hk + (size_t)(Nk - 1 - j) * d;\n                    for (int k = 0; k < d; ++k) o[k] += P[j] * v[k];\n                }\n            }\n        free(P);\n    }\n    return err;\n}\n\nint oracle_fwd("),
 ]
 
 # The pins each mutant is run against (all cheap).
@@ -44,6 +49,9 @@ PIN_CALLS = [
     ("identities_causal", lambda gd: pins.test_gradient_identities("causal")),
     ("sdpa_causal", lambda gd: pins.test_against_torch_sdpa_fp64("causal", (1, 3, 128, 64))),
     ("sdpa_block", lambda gd: pins.test_against_torch_sdpa_fp64("block", (2, 2, 200, 32))),
+    ("cross_suffix", lambda gd: pins.test_cross_causal_suffix_equals_square_problem()),
+    ("cross_more_queries", lambda gd: pins.test_cross_causal_more_queries_than_keys()),
+    ("cross_block", lambda gd: pins.test_cross_block_mask_is_query_blocks_by_key_blocks()),
 ]
 
 

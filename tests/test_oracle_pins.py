@@ -278,3 +278,128 @@ def test_bf16_inputs_are_widened_exactly():
     a = oracle._f64(x["Q"])
     np.testing.assert_array_equal(a, x["Q"].float().double().numpy())
     assert x["Q"].dtype == torch.bfloat16
+
+
+# ------------------------------------ queries and keys of different counts --
+# Causal with Nq != Nk is aligned at the bottom right: query i sees key j iff
+# j <= i + (Nk - Nq) (the last query sees every key).
+
+def test_cross_causal_suffix_equals_square_problem():
+    """The last Nq queries of a square causal problem over Nk keys see exactly
+    what Nq queries see against those Nk keys: O, LSE and dQ agree, and with
+    dO zero on the other rows so do dK and dV."""
+    Nk, Nq, d, scale = 40, 13, 8, 0.4
+    q, k, v, do = (rnd((2, Nk, d), s) for s in (60, 61, 62, 63))
+    do_sq = do.copy()
+    do_sq[:, : Nk - Nq] = 0.0
+    sq = oracle.bwd(q, k, v, do_sq, "causal", None, scale)
+    cr = oracle.bwd(q[:, Nk - Nq:], k, v, do[:, Nk - Nq:], "causal", None, scale)
+    for name in ("O", "dQ"):
+        np.testing.assert_allclose(cr[name], sq[name][:, Nk - Nq:], atol=1e-13, err_msg=name)
+    np.testing.assert_allclose(cr["LSE"], sq["LSE"][:, Nk - Nq:], atol=1e-13)
+    for name in ("dK", "dV"):
+        np.testing.assert_allclose(cr[name], sq[name], atol=1e-13, err_msg=name)
+
+
+def test_cross_causal_more_queries_than_keys():
+    """Nq > Nk: the first Nq - Nk queries see no key (O = 0, LSE = -inf, no
+    gradient); the last Nk form the square causal problem over the keys."""
+    Nk, Nq, d, scale = 9, 20, 6, 0.5
+    q, do = rnd((1, Nq, d), 64), rnd((1, Nq, d), 65)
+    k, v = rnd((1, Nk, d), 66), rnd((1, Nk, d), 67)
+    cr = oracle.bwd(q, k, v, do, "causal", None, scale)
+    sq = oracle.bwd(q[:, Nq - Nk:], k, v, do[:, Nq - Nk:], "causal", None, scale)
+    e = Nq - Nk
+    assert np.all(cr["O"][:, :e] == 0.0) and np.all(cr["dQ"][:, :e] == 0.0)
+    assert np.all(np.isneginf(cr["LSE"][:, :e]))
+    for name in ("O", "dQ"):
+        np.testing.assert_allclose(cr[name][:, e:], sq[name], atol=1e-13, err_msg=name)
+    for name in ("dK", "dV"):
+        np.testing.assert_allclose(cr[name], sq[name], atol=1e-13, err_msg=name)
+
+
+@pytest.mark.parametrize("Nk", [1, 5, 300])
+def test_single_query_sees_every_key(Nk):
+    """Decode shape: one query against Nk keys; under bottom-right causal it
+    sees every key, so causal equals no mask."""
+    d, scale = 16, 0.25
+    q, do = rnd((3, 1, d), 68), rnd((3, 1, d), 69)
+    k, v = rnd((3, Nk, d), 70), rnd((3, Nk, d), 71)
+    a = oracle.bwd(q, k, v, do, "causal", None, scale)
+    b = oracle.bwd(q, k, v, do, "none", None, scale)
+    for name in ("O", "LSE", "dQ", "dK", "dV"):
+        np.testing.assert_allclose(a[name], b[name], atol=0, err_msg=name)
+
+
+@pytest.mark.parametrize("kind", ["none", "causal"])
+@pytest.mark.parametrize("Nq,Nk", [(1, 300), (77, 160), (160, 77)])
+def test_cross_against_torch_sdpa_fp64(kind, Nq, Nk):
+    """PyTorch's fp64 attention with autograd; causal through a boolean mask
+    from torch.tril with the diagonal shifted by Nk - Nq."""
+    d, scale = 32, 0.2
+    g = torch.Generator().manual_seed(72)
+    q, do = (torch.randn((1, 2, Nq, d), generator=g, dtype=torch.float64) for _ in range(2))
+    k, v = (torch.randn((1, 2, Nk, d), generator=g, dtype=torch.float64) for _ in range(2))
+    qt, kt, vt = (t.clone().requires_grad_(True) for t in (q, k, v))
+    am = None
+    if kind == "causal":
+        am = torch.ones(Nq, Nk, dtype=torch.bool).tril(diagonal=Nk - Nq)
+    if am is not None and not am.any(dim=1).all():
+        # PyTorch returns NaN for a row with no visible key; compare the rest
+        live = am.any(dim=1)
+    else:
+        live = torch.ones(Nq, dtype=torch.bool)
+    out = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=am, scale=scale)
+    (out[:, :, live] * do[:, :, live]).sum().backward()
+    gr = oracle.bwd(q, k, v, do * live[None, None, :, None], kind, None, scale)
+    np.testing.assert_allclose(gr["O"][:, :, live.numpy()], out.detach()[:, :, live].numpy(), atol=1e-10)
+    for name, t in (("dQ", qt), ("dK", kt), ("dV", vt)):
+        ref = t.grad.numpy()
+        got = gr[name]
+        if name == "dQ":
+            ref, got = ref[:, :, live.numpy()], got[:, :, live.numpy()]
+        np.testing.assert_allclose(got, ref, atol=1e-10, err_msg=name)
+
+
+def test_cross_block_mask_is_query_blocks_by_key_blocks():
+    """A block mask over Nq != Nk is ceil(Nq/b) x ceil(Nk/b): all ones equals
+    no mask, and a mask keeping key block 2 only equals attention over the
+    keys of that block."""
+    Nq, Nk, d, b, scale = 200, 330, 8, 64, 0.3
+    q, k, v = rnd((2, Nq, d), 73), rnd((2, Nk, d), 74), rnd((2, Nk, d), 75)
+    nbq, nbk = -(-Nq // b), -(-Nk // b)
+    ones = np.ones((nbq, nbk), np.uint8)
+    O1, L1 = oracle.fwd(q, k, v, "block", ones, scale, block=b)
+    O0, L0 = oracle.fwd(q, k, v, "none", None, scale)
+    np.testing.assert_allclose(O1, O0, atol=0)
+    np.testing.assert_allclose(L1, L0, atol=0)
+    col = np.zeros((nbq, nbk), np.uint8)
+    col[:, 2] = 1
+    O2, L2 = oracle.fwd(q, k, v, "block", col, scale, block=b)
+    O3, L3 = oracle.fwd(q, k[:, 2 * b:3 * b], v[:, 2 * b:3 * b], "none", None, scale)
+    np.testing.assert_allclose(O2, O3, atol=1e-14)
+    np.testing.assert_allclose(L2, L3, atol=1e-14)
+
+
+def test_cross_gradients_by_finite_differences():
+    Nq, Nk, d, scale, h = 5, 9, 4, 0.6, 1e-6
+    q, do = rnd((1, Nq, d), 76), rnd((1, Nq, d), 77)
+    k, v = rnd((1, Nk, d), 78), rnd((1, Nk, d), 79)
+
+    def loss(q_, k_, v_):
+        O, _ = oracle.fwd(q_, k_, v_, "causal", None, scale)
+        return float((O * do).sum())
+
+    g = oracle.bwd(q, k, v, do, "causal", None, scale)
+    for name, idx, n in (("dQ", 0, Nq), ("dK", 1, Nk), ("dV", 2, Nk)):
+        fd = np.zeros((n, d))
+        for i in range(n):
+            for c in range(d):
+                args_p = [q.copy(), k.copy(), v.copy()]
+                args_m = [q.copy(), k.copy(), v.copy()]
+                args_p[idx][0, i, c] += h
+                args_m[idx][0, i, c] -= h
+                fd[i, c] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        ref = g[name][0]
+        err = np.abs(fd - ref).max() / max(1e-30, np.abs(ref).max())
+        assert err < 1e-6, (name, err)
