@@ -35,6 +35,10 @@ SIGNATURES = {
     "fa_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fa_bwd_stage": (_i, [_i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp, _vp,
                           _sz, _vp]),
+    "fa_fwd_qk": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp]),
+    "fa_bwd_workspace_size_qk": (_sz, [_i, _i, _i, _i, _i]),
+    "fa_bwd_qk": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp, _vp, _sz,
+                       _vp]),
     "fa_bwd_static_workspace": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp,
                                      _vp, _vp]),
     "fa_device_status": (_i, [_vp]),
@@ -97,42 +101,64 @@ def _check_qkv(*ts):
             raise FAError(1, "tensors must be contiguous bf16 CUDA tensors [B, H, N, d]")
 
 
+def _nk(Q, K, V):
+    """Key count of K, V [B,H,Nk,d] (heads and head dimension as Q's)."""
+    if K.shape != V.shape or K.shape[:2] != Q.shape[:2] or K.shape[3] != Q.shape[3]:
+        raise FAError(1, "K and V must be [B, H, Nk, d] with Q's B, H and d")
+    return K.shape[2]
+
+
 def fwd(Q, K, V, mask="none", block_mask=None, scale=None, O=None, LSE=None, stream=None):
-    """O [B,H,N,d] bf16 and LSE [B,H,N] fp32 (natural log)."""
+    """O [B,H,Nq,d] bf16 and LSE [B,H,Nq] fp32 (natural log); K, V are
+    [B,H,Nk,d] (Nk may differ from Nq: fa_fwd_qk)."""
     _check_qkv(Q, K, V)
     B, H, N, d = Q.shape
+    Nk = _nk(Q, K, V)
     scale = d ** -0.5 if scale is None else float(scale)
     kind, mptr = _mask(mask, block_mask)
     if O is None:
         O = torch.empty_like(Q)
     if LSE is None:
         LSE = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
-    _check(lib().fa_fwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, H, N, d, kind, mptr, scale,
-                        O.data_ptr(), LSE.data_ptr(), _stream(stream)), "fa_fwd")
+    if Nk == N:
+        _check(lib().fa_fwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, H, N, d, kind, mptr, scale,
+                            O.data_ptr(), LSE.data_ptr(), _stream(stream)), "fa_fwd")
+    else:
+        _check(lib().fa_fwd_qk(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, H, N, Nk, d, kind, mptr, scale,
+                               O.data_ptr(), LSE.data_ptr(), _stream(stream)), "fa_fwd_qk")
     return O, LSE
 
 
-def bwd_workspace_size(B, H, N, d) -> int:
-    return int(lib().fa_bwd_workspace_size(B, H, N, d))
+def bwd_workspace_size(B, H, N, d, Nk=None) -> int:
+    if Nk is None:
+        return int(lib().fa_bwd_workspace_size(B, H, N, d))
+    return int(lib().fa_bwd_workspace_size_qk(B, H, N, Nk, d))
 
 
 def bwd(Q, K, V, O, dO, LSE, mask="none", block_mask=None, scale=None, dQ=None, dK=None, dV=None,
         workspace=None, stream=None):
-    """dQ, dK, dV [B,H,N,d] bf16."""
+    """dQ [B,H,Nq,d], dK, dV [B,H,Nk,d] bf16 (Nk may differ from Nq: fa_bwd_qk)."""
     _check_qkv(Q, K, V, O, dO)
     B, H, N, d = Q.shape
+    Nk = _nk(Q, K, V)
     scale = d ** -0.5 if scale is None else float(scale)
     kind, mptr = _mask(mask, block_mask)
     dQ = torch.empty_like(Q) if dQ is None else dQ
     dK = torch.empty_like(K) if dK is None else dK
     dV = torch.empty_like(V) if dV is None else dV
-    ws = bwd_workspace_size(B, H, N, d)
+    ws = bwd_workspace_size(B, H, N, d, Nk)
     if workspace is None:
         workspace = torch.empty(ws, dtype=torch.uint8, device=Q.device)
-    _check(lib().fa_bwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(), dO.data_ptr(),
-                        LSE.data_ptr(), B, H, N, d, kind, mptr, scale, dQ.data_ptr(), dK.data_ptr(),
-                        dV.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)),
-           "fa_bwd")
+    if Nk == N:
+        _check(lib().fa_bwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(), dO.data_ptr(),
+                            LSE.data_ptr(), B, H, N, d, kind, mptr, scale, dQ.data_ptr(), dK.data_ptr(),
+                            dV.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)),
+               "fa_bwd")
+    else:
+        _check(lib().fa_bwd_qk(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(), dO.data_ptr(),
+                               LSE.data_ptr(), B, H, N, Nk, d, kind, mptr, scale, dQ.data_ptr(), dK.data_ptr(),
+                               dV.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)),
+               "fa_bwd_qk")
     return dQ, dK, dV
 
 

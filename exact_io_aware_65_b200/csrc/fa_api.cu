@@ -79,10 +79,14 @@ using namespace fa;
 
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-static fa_status check_common(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+static bool sizes_supported(long long bh, int N) {
+  return bh <= (1ll << 30) && N <= (1 << 30) && bh * (long long)N <= (1ll << 40);
+}
+
+static fa_status check_common(const void* Q, const void* K, const void* V, int B, int H, int N, int Nk, int d,
                               int mask_kind, const uint8_t* block_mask, float scale, Problem* p) {
   if (!Q || !K || !V) return FA_ERR_INVALID_ARG;
-  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || N <= 0 || Nk <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (mask_kind != FA_MASK_NONE && mask_kind != FA_MASK_CAUSAL && mask_kind != FA_MASK_BLOCK)
     return FA_ERR_INVALID_ARG;
@@ -90,10 +94,12 @@ static fa_status check_common(const void* Q, const void* K, const void* V, int B
   if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   const long long bh = (long long)B * H;
-  if (bh > (1ll << 30) || N > (1 << 30) || bh * (long long)N > (1ll << 40)) return FA_ERR_UNSUPPORTED;
-  p->B = B; p->H = H; p->N = N; p->d = d;
+  if (!sizes_supported(bh, N) || !sizes_supported(bh, Nk)) return FA_ERR_UNSUPPORTED;
+  p->B = B; p->H = H; p->N = N; p->Nk = Nk; p->d = d;
   p->BH = (int)bh;
   p->nq = (N + 127) / 128;
+  p->nk = (Nk + 127) / 128;
+  p->off = Nk - N;
   p->mask_kind = mask_kind;
   p->block_mask = mask_kind == FA_MASK_BLOCK ? block_mask : nullptr;
   p->scale = scale;
@@ -103,28 +109,37 @@ static fa_status check_common(const void* Q, const void* K, const void* V, int B
 
 extern "C" {
 
-fa_status fa_fwd(const void* Q, const void* K, const void* V, int B, int H, int N, int d, int mask_kind,
-                 const uint8_t* block_mask, float scale, void* O, float* LSE, void* stream) {
+fa_status fa_fwd_qk(const void* Q, const void* K, const void* V, int B, int H, int Nq, int Nk, int d,
+                    int mask_kind, const uint8_t* block_mask, float scale, void* O, float* LSE, void* stream) {
   Problem p;
-  fa_status st = check_common(Q, K, V, B, H, N, d, mask_kind, block_mask, scale, &p);
+  fa_status st = check_common(Q, K, V, B, H, Nq, Nk, d, mask_kind, block_mask, scale, &p);
   if (st != FA_OK) return st;
   if (!O || !LSE || !aligned(O, 16) || !aligned(LSE, 4)) return FA_ERR_INVALID_ARG;
   return launch_fwd(p, Q, K, V, O, LSE, (cudaStream_t)stream);
 }
 
+fa_status fa_fwd(const void* Q, const void* K, const void* V, int B, int H, int N, int d, int mask_kind,
+                 const uint8_t* block_mask, float scale, void* O, float* LSE, void* stream) {
+  return fa_fwd_qk(Q, K, V, B, H, N, N, d, mask_kind, block_mask, scale, O, LSE, stream);
+}
+
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || (d != 64 && d != 128)) return 0;
-  const long long bh = (long long)B * H;
-  if (bh > (1ll << 30) || N > (1 << 30) || bh * (long long)N > (1ll << 40)) return 0;
+  if (!sizes_supported((long long)B * H, N)) return 0;
   return bwd_workspace_bytes(B, H, N, d);
 }
 
+size_t fa_bwd_workspace_size_qk(int B, int H, int Nq, int Nk, int d) {
+  if (Nk <= 0 || !sizes_supported((long long)B * H, Nk)) return 0;
+  return fa_bwd_workspace_size(B, H, Nq, d);  // the workspace is per query row
+}
+
 static fa_status bwd_common(int stage, const void* Q, const void* K, const void* V, const void* O, const void* dO,
-                            const float* LSE, int B, int H, int N, int d, int mask_kind, const uint8_t* block_mask,
-                            float scale, void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes,
-                            void* stream) {
+                            const float* LSE, int B, int H, int N, int Nk, int d, int mask_kind,
+                            const uint8_t* block_mask, float scale, void* dQ, void* dK, void* dV, void* workspace,
+                            size_t workspace_bytes, void* stream) {
   Problem p;
-  fa_status st = check_common(Q, K, V, B, H, N, d, mask_kind, block_mask, scale, &p);
+  fa_status st = check_common(Q, K, V, B, H, N, Nk, d, mask_kind, block_mask, scale, &p);
   if (st != FA_OK) return st;
   if (!O || !dO || !LSE || !dQ || !dK || !dV) return FA_ERR_INVALID_ARG;
   if (!aligned(O, 16) || !aligned(dO, 16) || !aligned(LSE, 4) || !aligned(dQ, 16) || !aligned(dK, 16) ||
@@ -138,7 +153,14 @@ static fa_status bwd_common(int stage, const void* Q, const void* K, const void*
 fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
                  int B, int H, int N, int d, int mask_kind, const uint8_t* block_mask, float scale, void* dQ,
                  void* dK, void* dV, void* workspace, size_t workspace_bytes, void* stream) {
-  return bwd_common(-1, Q, K, V, O, dO, LSE, B, H, N, d, mask_kind, block_mask, scale, dQ, dK, dV, workspace,
+  return bwd_common(-1, Q, K, V, O, dO, LSE, B, H, N, N, d, mask_kind, block_mask, scale, dQ, dK, dV, workspace,
+                    workspace_bytes, stream);
+}
+
+fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                    int B, int H, int Nq, int Nk, int d, int mask_kind, const uint8_t* block_mask, float scale,
+                    void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_common(-1, Q, K, V, O, dO, LSE, B, H, Nq, Nk, d, mask_kind, block_mask, scale, dQ, dK, dV, workspace,
                     workspace_bytes, stream);
 }
 
@@ -147,7 +169,7 @@ fa_status fa_bwd_stage(int stage, const void* Q, const void* K, const void* V, c
                        float scale, void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes,
                        void* stream) {
   if (stage < 0 || stage > 2) return FA_ERR_INVALID_ARG;
-  return bwd_common(stage, Q, K, V, O, dO, LSE, B, H, N, d, mask_kind, block_mask, scale, dQ, dK, dV, workspace,
+  return bwd_common(stage, Q, K, V, O, dO, LSE, B, H, N, N, d, mask_kind, block_mask, scale, dQ, dK, dV, workspace,
                     workspace_bytes, stream);
 }
 

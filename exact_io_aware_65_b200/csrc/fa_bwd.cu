@@ -37,6 +37,7 @@
 // dP^T columns for d = 128 (the next dP^T waits for the drain) and has two
 // buffers at [384,448) and [448,512) for d = 64.
 #include <cuda_bf16.h>
+#include <limits.h>
 #include <math.h>
 
 #include "fa_internal.h"
@@ -207,7 +208,8 @@ struct Cfg {
 };
 
 struct Params {
-  int BH, N, Npad, nq, n_items, mask_kind;
+  int BH, N, Npad, nq, n_items, mask_kind;  // N, Npad, nq: query rows, padded rows, tiles
+  int Nk, nk, off;  // key rows and tiles; causal: query i sees keys j <= i + off
   const uint8_t* block_mask;
   float scale, scale_log2;
   const float* Dw;
@@ -231,7 +233,7 @@ struct Item {
 // (under a causal mask they meet the most query tiles and run longest).
 
 __device__ __forceinline__ Item item_at(const Params& p, int idx) {
-  const int per_group = p.group * p.nq;
+  const int per_group = p.group * p.nk;
   const int g = idx / per_group, r = idx % per_group;
   const int gsize = min(p.group, p.BH - g * p.group);
   Item it;
@@ -243,12 +245,16 @@ __device__ __forceinline__ Item item_at(const Params& p, int idx) {
 constexpr int RING = 4;     // depth of the item ring the producer fills
 constexpr int CONSUMERS = 13;  // MMA warp + 8 softmax warps + 4 drain warps
 
-// Next query tile >= i that attends to key tile j (nq if none).
+// Next query tile >= i that attends to key tile j (nq if none).  Causal:
+// the rows that see some key of tile j are those >= j * BK - off.
 __device__ __forceinline__ int next_q(const Params& p, int j, int i) {
-  if (p.mask_kind == FA_MASK_CAUSAL) return i < j ? j : i;
+  if (p.mask_kind == FA_MASK_CAUSAL) {
+    const int first = max(0, j * BK - p.off) / BQ;
+    return i < first ? min(first, p.nq) : i;
+  }
   if (p.mask_kind == FA_MASK_BLOCK) {
     for (; i < p.nq; ++i)
-      if (__ldg(p.block_mask + (size_t)i * p.nq + j)) return i;
+      if (__ldg(p.block_mask + (size_t)i * p.nk + j)) return i;
   }
   return i;
 }
@@ -569,10 +575,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // producer with Q and dO (same stage index as the MMA warp uses)
         const float* sL = sLD + ((s_cnt - 1) % C::NST) * 256 + hf * 64;
         const float* sD = sL + 128;
-        const bool key_live = key < p.N;
-        const bool diag = p.mask_kind == FA_MASK_CAUSAL && i == it.j;
-        // element masks only on the causal diagonal and a ragged last key tile
-        const bool masked = diag || (it.j + 1) * BK > p.N;
+        // causal: query row q sees this key iff key <= q + off; some pair in
+        // the tile is hidden iff its last key exceeds its first row's limit
+        const bool cmask = p.mask_kind == FA_MASK_CAUSAL && it.j * BK + BK - 1 > i * BQ + p.off;
+        // element masks only where the causal boundary or a ragged last key
+        // tile crosses the tile: column c of this thread is hidden iff
+        // c < kq, kq folding both tests (a missing key hides every column)
+        const bool masked = cmask || (it.j + 1) * BK > p.Nk;
+        const int kq = key >= p.Nk ? INT_MAX : (cmask ? key - (i * BQ + hf * 64 + p.off) : INT_MIN);
         // ---- P^T = exp2(S^T * scale * log2e - LSE_i * log2e), kept packed
         // as bf16 pairs (the form the dV product reads) for the dS step too.
         uint32_t pk[32];
@@ -594,7 +604,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (masked) {
 #pragma unroll
               for (int e = 0; e < 4; ++e)
-                if (!key_live || (diag && hf * 64 + 4 * u + e < kr)) pv[e] = 0.0f;
+                if (kq > 4 * u + e) pv[e] = 0.0f;
             }
             pk[2 * u] = pack_bf16x2(pv[0], pv[1]);
             pk[2 * u + 1] = pack_bf16x2(pv[2], pv[3]);
@@ -660,8 +670,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       ++dk_cnt;
       tc_fence_after();
-      const bool store = key < p.N;
-      const size_t gbase = ((size_t)it.bh * p.N + key) * D;
+      const bool store = key < p.Nk;
+      const size_t gbase = ((size_t)it.bh * p.Nk + key) * D;
 #pragma unroll
       for (int g = 0; g < 2; ++g) {  // 0: dV, 1: dK
         const float mul = g == 0 ? 1.0f : p.scale;
@@ -813,7 +823,10 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     p.N = pr.N;
     p.Npad = Npad;
     p.nq = pr.nq;
-    p.n_items = pr.BH * pr.nq;
+    p.Nk = pr.Nk;
+    p.nk = pr.nk;
+    p.off = pr.off;
+    p.n_items = pr.BH * pr.nk;
     p.mask_kind = pr.mask_kind;
     p.block_mask = pr.block_mask;
     p.scale = pr.scale;
@@ -850,8 +863,8 @@ fa_status launch_bwd(const Problem& pr, const void* Q, const void* K, const void
   uint32_t* st = status_word();
   if (!st) return FA_ERR_CUDA;
   CUtensorMap mQ, mK, mV, mdO;
-  if (!make_map_bf16(&mQ, Q, pr.BH, pr.N, pr.d, 128) || !make_map_bf16(&mK, K, pr.BH, pr.N, pr.d, 128) ||
-      !make_map_bf16(&mV, V, pr.BH, pr.N, pr.d, 128) || !make_map_bf16(&mdO, dO, pr.BH, pr.N, pr.d, 128))
+  if (!make_map_bf16(&mQ, Q, pr.BH, pr.N, pr.d, 128) || !make_map_bf16(&mK, K, pr.BH, pr.Nk, pr.d, 128) ||
+      !make_map_bf16(&mV, V, pr.BH, pr.Nk, pr.d, 128) || !make_map_bf16(&mdO, dO, pr.BH, pr.N, pr.d, 128))
     return FA_ERR_CUDA;
   if (pr.d == 64) return launch_bwd_d<64>(pr, mQ, mK, mV, mdO, O, dO, LSE, dQ, dK, dV, workspace, s, st, stage);
   return launch_bwd_d<128>(pr, mQ, mK, mV, mdO, O, dO, LSE, dQ, dK, dV, workspace, s, st, stage);

@@ -74,7 +74,8 @@ struct Cfg {
 };
 
 struct Params {
-  int BH, N, nq, n_pairs, n_items, mask_kind;
+  int BH, N, nq, n_pairs, n_items, mask_kind;  // N, nq: query rows and tiles
+  int Nk, nk, off;  // key rows and tiles; causal: query i sees keys j <= i + off
   int group;  // heads per scheduling group
   const uint8_t* block_mask;
   float scale_log2;
@@ -108,16 +109,26 @@ __device__ __forceinline__ Item item_at(const Params& p, int idx) {
   return it;
 }
 
+// Last key a query row of tile qt may see under the causal mask (the tile's
+// last real row, shifted by the alignment; negative: none).
+__device__ __forceinline__ int causal_last_key(const Params& p, int qt) {
+  return min(qt * BM + BM - 1, p.N - 1) + p.off;
+}
+
 // Does query tile qt attend to key tile j?
 __device__ __forceinline__ bool member(const Params& p, int qt, int j) {
-  if (p.mask_kind == FA_MASK_CAUSAL) return j <= qt;
-  if (p.mask_kind == FA_MASK_BLOCK) return __ldg(p.block_mask + (size_t)qt * p.nq + j) != 0;
+  if (p.mask_kind == FA_MASK_CAUSAL) return j * BN <= causal_last_key(p, qt);
+  if (p.mask_kind == FA_MASK_BLOCK) return __ldg(p.block_mask + (size_t)qt * p.nk + j) != 0;
   return true;
 }
 
+// One past the last key tile either query tile of the item may need.
 __device__ __forceinline__ int kv_end(const Params& p, const Item& it) {
-  if (p.mask_kind == FA_MASK_CAUSAL) return (it.has1 ? it.q1 : it.q0) + 1;
-  return p.nq;
+  if (p.mask_kind == FA_MASK_CAUSAL) {
+    const int last = causal_last_key(p, it.has1 ? it.q1 : it.q0);
+    return last < 0 ? 0 : min(p.nk, last / BN + 1);
+  }
+  return p.nk;
 }
 
 // Next key tile >= j needed by either query tile of the item (kv_end if none).
@@ -425,9 +436,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         float x[BN];
 #pragma unroll
         for (int c = 0; c < BN; ++c) x[c] = __uint_as_float(sraw[c]);
+        // valid columns [0, lim): keys that exist and, under the causal mask,
+        // keys <= row + off
         const int key0 = j * BN;
-        const bool diag = p.mask_kind == FA_MASK_CAUSAL && j == qt;
-        const int lim = min(diag ? r + 1 : BN, p.N - key0);  // valid columns: [0, lim)
+        int lim = min(BN, p.Nk - key0);
+        if (p.mask_kind == FA_MASK_CAUSAL) lim = max(0, min(lim, row + p.off + 1 - key0));
         if (lim < BN) {
 #pragma unroll
           for (int c = 0; c < BN; ++c)
@@ -532,13 +545,16 @@ fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void
   uint32_t* st = status_word();
   if (!st) return FA_ERR_CUDA;
   CUtensorMap mQ, mK, mV;
-  if (!make_map_bf16(&mQ, Q, pr.BH, pr.N, pr.d, fwd::BM) || !make_map_bf16(&mK, K, pr.BH, pr.N, pr.d, fwd::BN) ||
-      !make_map_bf16(&mV, V, pr.BH, pr.N, pr.d, fwd::BN))
+  if (!make_map_bf16(&mQ, Q, pr.BH, pr.N, pr.d, fwd::BM) || !make_map_bf16(&mK, K, pr.BH, pr.Nk, pr.d, fwd::BN) ||
+      !make_map_bf16(&mV, V, pr.BH, pr.Nk, pr.d, fwd::BN))
     return FA_ERR_CUDA;
   fwd::Params p;
   p.BH = pr.BH;
   p.N = pr.N;
   p.nq = pr.nq;
+  p.Nk = pr.Nk;
+  p.nk = pr.nk;
+  p.off = pr.off;
   p.n_pairs = (pr.nq + 1) / 2;
   p.n_items = p.n_pairs * pr.BH;
   p.group = pr.BH < 8 ? pr.BH : 8;

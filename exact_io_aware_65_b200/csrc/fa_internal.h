@@ -11,11 +11,13 @@ namespace fa {
 
 // Problem description after validation.
 struct Problem {
-  int B, H, N, d;
-  int BH;        // B * H
-  int nq;        // ceil(N / 128): query tiles == key tiles (self-attention)
+  int B, H, N, d;  // N: query rows
+  int Nk;          // key rows (N for self-attention)
+  int BH;          // B * H
+  int nq, nk;      // ceil(N / 128) query tiles, ceil(Nk / 128) key tiles
+  int off;         // Nk - N: causal alignment (query i sees keys j <= i + off)
   int mask_kind;
-  const uint8_t* block_mask;  // device [nq, nq] or nullptr
+  const uint8_t* block_mask;  // device [nq, nk] or nullptr
   float scale;
   float scale_log2;  // scale * log2(e), computed in double and rounded once
 };

@@ -103,6 +103,30 @@ fa_status fa_bwd_stage(int stage, const void* Q, const void* K, const void* V, c
                        const uint8_t* block_mask, float scale, void* dQ, void* dK, void* dV,
                        void* workspace, size_t workspace_bytes, void* stream);
 
+/* Queries and keys of different counts (cross-attention, or a block of new
+ * queries against a longer key/value history).  Same as fa_fwd, fa_bwd and
+ * fa_bwd_workspace_size, which are these with Nq = Nk = N, except:
+ *   - Q, O, dO, dQ are [B,H,Nq,d] and LSE [B,H,Nq]; K, V, dK, dV are
+ *     [B,H,Nk,d].  Nq, Nk >= 1, any values (not multiples of 128).
+ *   - FA_MASK_CAUSAL is aligned at the bottom right: query i sees key j iff
+ *     j <= i + (Nk - Nq), so the last query sees every key (for Nq = Nk this
+ *     is j <= i).  The pages do not treat Nq != Nk; this alignment keeps a
+ *     suffix of the queries' outputs equal to those of the full square
+ *     problem.  With Nq > Nk the first Nq - Nk queries see nothing: O = 0,
+ *     LSE = -inf and no gradient, as for any row that sees no key.
+ *   - FA_MASK_BLOCK takes a [ceil(Nq/128), ceil(Nk/128)] uint8 DEVICE grid
+ *     (query tiles by key tiles, 1 = keep).
+ *   - The workspace depends on Nq only.
+ * Errors as for fa_fwd / fa_bwd (Nk <= 0 is FA_ERR_INVALID_ARG). */
+fa_status fa_fwd_qk(const void* Q, const void* K, const void* V, int B, int H, int Nq, int Nk, int d,
+                    int mask_kind, const uint8_t* block_mask, float scale, void* O, float* LSE,
+                    void* stream);
+size_t fa_bwd_workspace_size_qk(int B, int H, int Nq, int Nk, int d);
+fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                    const float* LSE, int B, int H, int Nq, int Nk, int d, int mask_kind,
+                    const uint8_t* block_mask, float scale, void* dQ, void* dK, void* dV,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* Largest scratch, in bytes, that fa_bwd_static_workspace() can use: 64 MiB. */
 #define FA_BWD_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
 

@@ -91,6 +91,25 @@ def make_inputs(w: Workload, seed: int = 0, grad: bool = True) -> dict:
     return out
 
 
+def make_cross_inputs(B: int, H: int, Nq: int, Nk: int, d: int, mask: str, seed: int = 0) -> dict:
+    """Queries and keys of different counts: Q, dO [B,H,Nq,d] and K, V
+    [B,H,Nk,d], bf16 CPU, drawn like ``make_inputs`` in the order Q, K, V, dO;
+    ``mask`` a uint8 [ceil(Nq/128), ceil(Nk/128)] grid for kind "block"
+    (generator seed + 1, keep probability P_KEEP, no forced blocks), else
+    None."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    out = {}
+    for name, n in (("Q", Nq), ("K", Nk), ("V", Nk), ("dO", Nq)):
+        out[name] = torch.randn((B, H, n, d), generator=g, dtype=torch.float32).to(torch.bfloat16).contiguous()
+    if mask == "block":
+        gm = torch.Generator("cpu").manual_seed(seed + 1)
+        nbq, nbk = (Nq + BLOCK - 1) // BLOCK, (Nk + BLOCK - 1) // BLOCK
+        out["mask"] = (torch.rand(nbq, nbk, generator=gm) < P_KEEP).to(torch.uint8).contiguous()
+    else:
+        out["mask"] = None
+    return out
+
+
 def kept_blocks(w: Workload, mask: torch.Tensor | None) -> int:
     """Number of 128x128 (or ragged-edge) score tiles a query attends to, summed
     over query tiles.  Pure counting, used for FLOP accounting."""
