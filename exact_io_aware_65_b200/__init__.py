@@ -39,6 +39,8 @@ SIGNATURES = {
     "fa_bwd_workspace_size_qk": (_sz, [_i, _i, _i, _i, _i]),
     "fa_bwd_qk": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp, _vp, _sz,
                        _vp]),
+    "fa_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "fa_decode": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _sz, _vp]),
     "fa_bwd_static_workspace": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp,
                                      _vp, _vp]),
     "fa_device_status": (_i, [_vp]),
@@ -173,6 +175,29 @@ def bwd_stage(stage, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, mask="none", bl
                               dO.data_ptr(), LSE.data_ptr(), B, H, N, d, kind, mptr, scale, dQ.data_ptr(),
                               dK.data_ptr(), dV.data_ptr(), workspace.data_ptr(), workspace.numel(),
                               _stream(stream)), f"fa_bwd_stage({stage})")
+
+
+def decode(Q, K, V, mask="none", scale=None, O=None, LSE=None, workspace=None, stream=None):
+    """Decode against a KV cache: Q [B,H,Nq,d] (Nq <= 16) against K, V
+    [B,H,Nk,d]; returns O [B,H,Nq,d] bf16 and LSE [B,H,Nq] fp32."""
+    _check_qkv(Q, K, V)
+    B, H, N, d = Q.shape
+    Nk = _nk(Q, K, V)
+    scale = d ** -0.5 if scale is None else float(scale)
+    kind, _ = _mask(mask, None)
+    if O is None:
+        O = torch.empty_like(Q)
+    if LSE is None:
+        LSE = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_size(B, H, N, Nk, d), dtype=torch.uint8, device=Q.device)
+    _check(lib().fa_decode(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, H, N, Nk, d, kind, scale, O.data_ptr(),
+                           LSE.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)), "fa_decode")
+    return O, LSE
+
+
+def decode_workspace_size(B, H, Nq, Nk, d) -> int:
+    return int(lib().fa_decode_workspace_size(B, H, Nq, Nk, d))
 
 
 def device_status(stream=None) -> int:

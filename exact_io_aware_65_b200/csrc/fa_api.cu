@@ -173,6 +173,27 @@ fa_status fa_bwd_stage(int stage, const void* Q, const void* K, const void* V, c
                     workspace_bytes, stream);
 }
 
+size_t fa_decode_workspace_size(int B, int H, int Nq, int Nk, int d) {
+  if (B <= 0 || H <= 0 || Nq <= 0 || Nq > 16 || Nk <= 0 || (d != 64 && d != 128)) return 0;
+  const long long bh = (long long)B * H;
+  if (!sizes_supported(bh, Nk)) return 0;
+  return decode_workspace_bytes((int)bh, Nq, Nk, d);
+}
+
+fa_status fa_decode(const void* Q, const void* K, const void* V, int B, int H, int Nq, int Nk, int d, int mask_kind,
+                    float scale, void* O, float* LSE, void* workspace, size_t workspace_bytes, void* stream) {
+  if (mask_kind == FA_MASK_BLOCK) return FA_ERR_UNSUPPORTED;
+  Problem p;
+  fa_status st = check_common(Q, K, V, B, H, Nq, Nk, d, mask_kind, nullptr, scale, &p);
+  if (st != FA_OK) return st;
+  if (Nq > 16) return FA_ERR_UNSUPPORTED;
+  if (!O || !LSE || !aligned(O, 16) || !aligned(LSE, 4)) return FA_ERR_INVALID_ARG;
+  const size_t need = decode_workspace_bytes(p.BH, Nq, Nk, d);
+  if (need == 0) return FA_ERR_CUDA;
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FA_ERR_WORKSPACE;
+  return launch_decode(p, Q, K, V, O, LSE, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
 fa_status fa_device_status(void* stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return FA_ERR_CUDA;
   uint32_t v = 0, zero = 0;

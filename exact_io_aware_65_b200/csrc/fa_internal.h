@@ -43,6 +43,11 @@ fa_status launch_bwd(const Problem& p, const void* Q, const void* K, const void*
                      const void* dO, const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
                      cudaStream_t s, int stage);
 size_t bwd_workspace_bytes(int B, int H, int N, int d);
+// Decode (few queries, long key history): workspace for the split-key
+// partial results on the current device (0 on failure), and the launch.
+size_t decode_workspace_bytes(int BH, int Nq, int Nk, int d);
+fa_status launch_decode(const Problem& p, const void* Q, const void* K, const void* V, void* O, float* LSE,
+                        void* workspace, size_t workspace_bytes, cudaStream_t s);
 fa_status launch_selftest_wait(uint64_t timeout_ns, cudaStream_t s);
 fa_status launch_selftest_mma(const void* A, const void* B, float* C, int n, int k, int mode, cudaStream_t s);
 

@@ -127,6 +127,27 @@ fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, 
                     const uint8_t* block_mask, float scale, void* dQ, void* dK, void* dV,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* Decode: a few new queries per head against a long key/value history (a
+ * KV cache), forward only.  The same exact attention as fa_fwd_qk, computed
+ * by splitting the keys across the GPU and merging the partial softmax
+ * results by their running maxima and sums (log-sum-exp); meant for the
+ * shapes where fa_fwd_qk would leave most of the GPU idle.
+ * In:  Q [B,H,Nq,d] bf16 with 1 <= Nq <= 16; K, V [B,H,Nk,d] bf16, Nk >= 1;
+ *      mask_kind FA_MASK_NONE or FA_MASK_CAUSAL (bottom-right aligned as in
+ *      fa_fwd_qk: query i sees keys j <= i + (Nk - Nq)); scale > 0;
+ *      workspace (DEVICE, 256-byte aligned, at least
+ *      fa_decode_workspace_size() bytes, contents irrelevant on entry).
+ * Out: O [B,H,Nq,d] bf16, LSE [B,H,Nq] fp32, as fa_fwd_qk.  All DEVICE
+ *      pointers, 16-byte aligned (LSE 4).
+ * Errors: FA_ERR_INVALID_ARG (as fa_fwd_qk), FA_ERR_UNSUPPORTED (Nq > 16,
+ * d not 64 or 128, a block mask), FA_ERR_WORKSPACE, FA_ERR_CUDA.  The pages
+ * have no decode-specific algorithm; this is their tiling applied across
+ * the keys, with the running statistics combined at the end. */
+size_t fa_decode_workspace_size(int B, int H, int Nq, int Nk, int d);
+fa_status fa_decode(const void* Q, const void* K, const void* V, int B, int H, int Nq, int Nk, int d,
+                    int mask_kind, float scale, void* O, float* LSE, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
 /* Largest scratch, in bytes, that fa_bwd_static_workspace() can use: 64 MiB. */
 #define FA_BWD_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
 
