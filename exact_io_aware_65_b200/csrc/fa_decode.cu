@@ -216,6 +216,8 @@ __global__ void __launch_bounds__(THREADS, 2) partial_kernel(const Params p) {
           const int q = q0 + qi * qs;
           if (q < p.Nq) acc[qi] *= alpha[q];
         }
+        // unrolled so that the loads of several keys are in flight at once
+#pragma unroll 8
         for (int kk = 0; kk < rows; ++kk) {
           const float v = __bfloat162float(vc[kk * D]);
 #pragma unroll
