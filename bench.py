@@ -221,6 +221,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--vs-standard", action="store_true",
+                    help="time the fused forward against standard (materialising) attention instead")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.workload in DECODE_WORKLOADS:
@@ -228,6 +230,8 @@ def main():
     w = workloads.WORKLOADS[args.workload]
     if args.impl == "reference":
         return reference_arm(args, w)
+    if args.vs_standard:
+        return vs_standard_main(args, w)
 
     import exact_io_aware_65_b200 as fa
 
@@ -388,6 +392,63 @@ def main():
         dist.destroy_process_group()
     if status != 0:
         raise SystemExit(f"device status {status}: a bounded wait timed out")
+
+
+def vs_standard_main(args, w):
+    """Forward of the fused kernel against standard attention (S = QK^T and
+    P in HBM, cuBLAS products + the library's softmax) on the same workload
+    and GPU: the speed and memory ratios the pages quote, measured here."""
+    import exact_io_aware_65_b200 as fa
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    x = workloads.make_inputs(w, args.seed, grad=False)
+    Q, K, V = (x[n].to(dev) for n in ("Q", "K", "V"))
+    mask = x["mask"].to(dev) if x["mask"] is not None else None
+    O1, O2 = torch.empty_like(Q), torch.empty_like(Q)
+    L1 = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    L2 = torch.empty_like(L1)
+    std_ws_bytes = fa.standard_fwd_workspace_size(w.B, w.H, w.N, w.d)
+    ws = torch.empty(std_ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    runs = {"fused": lambda: fa.fwd(Q, K, V, w.mask, mask, w.scale, O=O1, LSE=L1, stream=stream),
+            "standard": lambda: fa.standard_fwd(Q, K, V, w.mask, mask, w.scale, O=O2, LSE=L2, workspace=ws,
+                                                stream=stream)}
+    ms = {}
+    clocks = ClockSampler(dev.index)
+    clocks.mark_start()
+    for name, run in runs.items():
+        for _ in range(args.warmup):
+            run()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            run()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms[name] = e0.elapsed_time(e1) / args.steps
+    clocks.mark_end()
+    status = fa.device_status()
+    max_diff = (O1.float() - O2.float()).abs().max().item()
+    fl = flops(w, x["mask"])["fwd"]
+    line = {
+        "metric": "forward time of standard (materialising) attention / fused forward, same workload and GPU",
+        "value": ms["standard"] / ms["fused"], "unit": "x", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w),
+        "fused": {"ms": ms["fused"], "tflops": fl / (ms["fused"] * 1e-3) / 1e12,
+                  "extra_device_bytes": 0},
+        "standard": {"ms": ms["standard"], "tflops_of_kept_work": fl / (ms["standard"] * 1e-3) / 1e12,
+                     "extra_device_bytes": std_ws_bytes,
+                     "note": "computes the whole N x N grid and masks it; S fp32 and P bf16 through HBM"},
+        "max_abs_diff_O": max_diff,
+        "clocks": clocks.result(),
+        "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+    if status != 0:
+        raise SystemExit(f"device status {status}")
 
 
 def decode_main(args, name, c):

@@ -41,6 +41,8 @@ SIGNATURES = {
                        _vp]),
     "fa_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "fa_decode": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _sz, _vp]),
+    "fa_standard_fwd_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "fa_standard_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp, _sz, _vp]),
     "fa_bwd_static_workspace": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp,
                                      _vp, _vp]),
     "fa_device_status": (_i, [_vp]),
@@ -194,6 +196,30 @@ def decode(Q, K, V, mask="none", scale=None, O=None, LSE=None, workspace=None, s
     _check(lib().fa_decode(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, H, N, Nk, d, kind, scale, O.data_ptr(),
                            LSE.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)), "fa_decode")
     return O, LSE
+
+
+def standard_fwd(Q, K, V, mask="none", block_mask=None, scale=None, O=None, LSE=None, workspace=None,
+                 stream=None):
+    """Standard (materialising) attention, the baseline: O [B,H,N,d] bf16 and
+    LSE [B,H,N] fp32, through an N x N score grid in HBM."""
+    _check_qkv(Q, K, V)
+    B, H, N, d = Q.shape
+    scale = d ** -0.5 if scale is None else float(scale)
+    kind, mptr = _mask(mask, block_mask)
+    if O is None:
+        O = torch.empty_like(Q)
+    if LSE is None:
+        LSE = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    if workspace is None:
+        workspace = torch.empty(standard_fwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=Q.device)
+    _check(lib().fa_standard_fwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, H, N, d, kind, mptr, scale,
+                                 O.data_ptr(), LSE.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                 _stream(stream)), "fa_standard_fwd")
+    return O, LSE
+
+
+def standard_fwd_workspace_size(B, H, N, d) -> int:
+    return int(lib().fa_standard_fwd_workspace_size(B, H, N, d))
 
 
 def decode_workspace_size(B, H, Nq, Nk, d) -> int:

@@ -42,7 +42,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     if not force and not _stale():
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *ARCH, *FLAGS, "-shared", "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
+    cmd = [NVCC, *ARCH, *FLAGS, "-shared", "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources(), "-ldl"]
     if ptxas_info:
         cmd[1:1] = ["-Xptxas", "-v"]
     if verbose:

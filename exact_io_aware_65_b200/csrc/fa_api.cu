@@ -194,6 +194,27 @@ fa_status fa_decode(const void* Q, const void* K, const void* V, int B, int H, i
   return launch_decode(p, Q, K, V, O, LSE, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
+size_t fa_standard_fwd_workspace_size(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || N > 16384 || (d != 64 && d != 128)) return 0;
+  const long long bh = (long long)B * H;
+  if (!sizes_supported(bh, N) || bh > (1 << 30) / 16) return 0;
+  return standard_workspace_bytes((int)bh, N);
+}
+
+fa_status fa_standard_fwd(const void* Q, const void* K, const void* V, int B, int H, int N, int d, int mask_kind,
+                          const uint8_t* block_mask, float scale, void* O, float* LSE, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  Problem p;
+  fa_status st = check_common(Q, K, V, B, H, N, N, d, mask_kind, block_mask, scale, &p);
+  if (st != FA_OK) return st;
+  if (N > 16384) return FA_ERR_UNSUPPORTED;
+  if (!O || !LSE || !aligned(O, 16) || !aligned(LSE, 4)) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_standard_fwd_workspace_size(B, H, N, d);
+  if (need == 0) return FA_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FA_ERR_WORKSPACE;
+  return launch_standard_fwd(p, Q, K, V, O, LSE, workspace, (cudaStream_t)stream);
+}
+
 fa_status fa_device_status(void* stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return FA_ERR_CUDA;
   uint32_t v = 0, zero = 0;

@@ -48,6 +48,11 @@ size_t bwd_workspace_bytes(int B, int H, int N, int d);
 size_t decode_workspace_bytes(int BH, int Nq, int Nk, int d);
 fa_status launch_decode(const Problem& p, const void* Q, const void* K, const void* V, void* O, float* LSE,
                         void* workspace, size_t workspace_bytes, cudaStream_t s);
+// Standard (materialising) attention, the baseline: workspace for S (fp32)
+// and P (bf16), and the launch.
+size_t standard_workspace_bytes(int BH, int N);
+fa_status launch_standard_fwd(const Problem& p, const void* Q, const void* K, const void* V, void* O, float* LSE,
+                              void* workspace, cudaStream_t s);
 fa_status launch_selftest_wait(uint64_t timeout_ns, cudaStream_t s);
 fa_status launch_selftest_mma(const void* A, const void* B, float* C, int n, int k, int mode, cudaStream_t s);
 

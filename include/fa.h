@@ -148,6 +148,23 @@ fa_status fa_decode(const void* Q, const void* K, const void* V, int B, int H, i
                     int mask_kind, float scale, void* O, float* LSE, void* workspace,
                     size_t workspace_bytes, void* stream);
 
+/* Standard (materialising) attention, forward only: the baseline the pages
+ * measure the method against, for speed and memory comparisons.  It writes
+ * S = scale Q K^T to HBM in fp32, reads it back for a masked row softmax
+ * that writes P in bf16, and reads P back for O = P V; the N x N grid makes
+ * two round trips through HBM and the workspace grows as N^2.  The two
+ * products are cuBLAS batched GEMMs (libcublas.so.12, opened at the first
+ * call); the softmax is the library's own kernel.
+ * In/out as fa_fwd (self-attention, N <= 16384, same masks and LSE
+ * convention); workspace (DEVICE, 256-byte aligned) of at least
+ * fa_standard_fwd_workspace_size() bytes: 6 * B * H * N^2 plus alignment.
+ * Errors as fa_fwd, plus FA_ERR_UNSUPPORTED (N > 16384), FA_ERR_WORKSPACE,
+ * and FA_ERR_CUDA when cuBLAS cannot be opened or fails. */
+size_t fa_standard_fwd_workspace_size(int B, int H, int N, int d);
+fa_status fa_standard_fwd(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                          int mask_kind, const uint8_t* block_mask, float scale, void* O, float* LSE,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
 /* Largest scratch, in bytes, that fa_bwd_static_workspace() can use: 64 MiB. */
 #define FA_BWD_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
 
