@@ -39,6 +39,8 @@ SIGNATURES = {
     "fa_bwd_workspace_size_qk": (_sz, [_i, _i, _i, _i, _i]),
     "fa_bwd_qk": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp, _vp, _sz,
                        _vp]),
+    "fa_bwd_qk_deterministic": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp,
+                                     _vp, _vp, _sz, _vp]),
     "fa_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "fa_decode": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _sz, _vp]),
     "fa_standard_fwd_workspace_size": (_sz, [_i, _i, _i, _i]),
@@ -140,7 +142,7 @@ def bwd_workspace_size(B, H, N, d, Nk=None) -> int:
 
 
 def bwd(Q, K, V, O, dO, LSE, mask="none", block_mask=None, scale=None, dQ=None, dK=None, dV=None,
-        workspace=None, stream=None):
+        workspace=None, stream=None, deterministic=False):
     """dQ [B,H,Nq,d], dK, dV [B,H,Nk,d] bf16 (Nk may differ from Nq: fa_bwd_qk)."""
     _check_qkv(Q, K, V, O, dO)
     B, H, N, d = Q.shape
@@ -153,7 +155,12 @@ def bwd(Q, K, V, O, dO, LSE, mask="none", block_mask=None, scale=None, dQ=None, 
     ws = bwd_workspace_size(B, H, N, d, Nk)
     if workspace is None:
         workspace = torch.empty(ws, dtype=torch.uint8, device=Q.device)
-    if Nk == N:
+    if deterministic:
+        _check(lib().fa_bwd_qk_deterministic(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(), dO.data_ptr(),
+                                             LSE.data_ptr(), B, H, N, Nk, d, kind, mptr, scale, dQ.data_ptr(),
+                                             dK.data_ptr(), dV.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                             _stream(stream)), "fa_bwd_qk_deterministic")
+    elif Nk == N:
         _check(lib().fa_bwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(), dO.data_ptr(),
                             LSE.data_ptr(), B, H, N, d, kind, mptr, scale, dQ.data_ptr(), dK.data_ptr(),
                             dV.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)),

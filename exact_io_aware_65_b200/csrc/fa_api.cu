@@ -137,9 +137,10 @@ size_t fa_bwd_workspace_size_qk(int B, int H, int Nq, int Nk, int d) {
 static fa_status bwd_common(int stage, const void* Q, const void* K, const void* V, const void* O, const void* dO,
                             const float* LSE, int B, int H, int N, int Nk, int d, int mask_kind,
                             const uint8_t* block_mask, float scale, void* dQ, void* dK, void* dV, void* workspace,
-                            size_t workspace_bytes, void* stream) {
+                            size_t workspace_bytes, void* stream, int deterministic = 0) {
   Problem p;
   fa_status st = check_common(Q, K, V, B, H, N, Nk, d, mask_kind, block_mask, scale, &p);
+  p.deterministic = deterministic;
   if (st != FA_OK) return st;
   if (!O || !dO || !LSE || !dQ || !dK || !dV) return FA_ERR_INVALID_ARG;
   if (!aligned(O, 16) || !aligned(dO, 16) || !aligned(LSE, 4) || !aligned(dQ, 16) || !aligned(dK, 16) ||
@@ -162,6 +163,14 @@ fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, 
                     void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_common(-1, Q, K, V, O, dO, LSE, B, H, Nq, Nk, d, mask_kind, block_mask, scale, dQ, dK, dV, workspace,
                     workspace_bytes, stream);
+}
+
+fa_status fa_bwd_qk_deterministic(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                                  const float* LSE, int B, int H, int Nq, int Nk, int d, int mask_kind,
+                                  const uint8_t* block_mask, float scale, void* dQ, void* dK, void* dV,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_common(-1, Q, K, V, O, dO, LSE, B, H, Nq, Nk, d, mask_kind, block_mask, scale, dQ, dK, dV, workspace,
+                    workspace_bytes, stream, 1);
 }
 
 fa_status fa_bwd_stage(int stage, const void* Q, const void* K, const void* V, const void* O, const void* dO,

@@ -57,9 +57,11 @@ __host__ __device__ constexpr size_t align256(size_t x) { return (x + 255) & ~si
 // accumulator is tiled: within each (head, 128-query tile) block the element
 // (query r, column c) sits at (c / 4) * 512 + r * 4 + c % 4, so that one warp
 // adding four columns of 32 consecutive query rows touches 512 contiguous
-// bytes.  `sched` is the work counter of the main kernel's dynamic scheduler.
+// bytes.  `sched` is the work counter of the main kernel's dynamic scheduler;
+// `turn` holds one counter per (head, query tile) for the deterministic
+// order of the dQ additions (how many key tiles have added their part).
 struct Workspace {
-  size_t dq_off, d_off, l2_off, sched_off, total;
+  size_t dq_off, d_off, l2_off, sched_off, turn_off, total;
 };
 __host__ __device__ inline Workspace workspace_layout(int BH, int Npad, int d) {
   Workspace w;
@@ -67,7 +69,8 @@ __host__ __device__ inline Workspace workspace_layout(int BH, int Npad, int d) {
   w.d_off = align256((size_t)BH * Npad * d * sizeof(float));
   w.l2_off = w.d_off + align256((size_t)BH * Npad * sizeof(float));
   w.sched_off = w.l2_off + align256((size_t)BH * Npad * sizeof(float));
-  w.total = w.sched_off + 256;
+  w.turn_off = w.sched_off + 256;
+  w.total = w.turn_off + align256((size_t)BH * (Npad / 128) * sizeof(uint32_t));
   return w;
 }
 
@@ -78,7 +81,8 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restri
                                                    const __nv_bfloat16* __restrict__ dO,
                                                    const float* __restrict__ LSE, float* __restrict__ Dw,
                                                    float* __restrict__ L2w, float* __restrict__ dq_acc,
-                                                   uint32_t* __restrict__ sched, int BH, int N, int Npad) {
+                                                   uint32_t* __restrict__ sched, uint32_t* __restrict__ turn,
+                                                   int BH, int N, int Npad) {
   constexpr int LPR = D / 8;
   if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0u;
   constexpr int RPW = 32 / LPR;
@@ -109,6 +113,7 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restri
     for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (r < total) {
       if (li == 0) {
+        if ((n & 127) == 0) turn[(size_t)bh * (Npad / 128) + n / 128] = 0u;
         Dw[r] = acc;
         float l2 = INFINITY;  // padding rows and rows that saw no key: P = 0
         if (real) {
@@ -216,6 +221,8 @@ struct Params {
   const float* L2w;
   float* dq_acc;
   uint32_t* sched;
+  uint32_t* turn;     // [BH, nq] dQ addition counters (deterministic mode)
+  int deterministic;  // add each query tile's dQ parts in key-tile order
   int group;  // heads per scheduling group
   __nv_bfloat16* dK;
   __nv_bfloat16* dV;
@@ -240,6 +247,53 @@ __device__ __forceinline__ Item item_at(const Params& p, int idx) {
   it.j = r / gsize;
   it.bh = g * p.group + r % gsize;
   return it;
+}
+
+// Deterministic dQ: the part of key tile j for query tile i is added only
+// once the key tiles before it that see query tile i have added theirs, so
+// every dQ element is summed in ascending key-tile order.  Its position in
+// that order:
+__device__ __forceinline__ uint32_t add_rank(const Params& p, int j, int i) {
+  if (p.mask_kind == FA_MASK_BLOCK) {
+    uint32_t r = 0;
+    for (int k = 0; k < j; ++k) r += __ldg(p.block_mask + (size_t)i * p.nk + k) != 0;
+    return r;
+  }
+  // no mask, or causal: a lower key tile is visible to every query row that
+  // sees a higher one, so all j tiles before this one see query tile i
+  return (uint32_t)j;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* a) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_add_gpu(uint32_t* a, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Bounded wait until *a == want (another CTA's release); false on timeout or
+// abort, with the CTA marked as aborting.
+__device__ bool wait_turn(const uint32_t* a, uint32_t want, const WaitCtx& w) {
+  uint64_t start = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (ld_acquire_gpu(a) == want) return true;
+    if ((it & 15u) == 15u) {
+      if (*w.abort_flag) return false;
+      const uint64_t now = globaltimer_ns();
+      if (start == 0) {
+        start = now;
+      } else if (now - start > w.timeout_ns) {
+        *w.abort_flag = 1;
+        atomicCAS(w.status, FA_DEV_OK, FA_DEV_ERR_TIMEOUT);
+        return false;
+      }
+    }
+    __nanosleep(64);
+  }
 }
 
 constexpr int RING = 4;     // depth of the item ring the producer fills
@@ -755,11 +809,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mbar_arrive(&dq_staged[h]);
           if (leader) {
             ok = mbar_wait(&dq_staged[h], dq_iter & 1, w);
+            uint32_t* turn = p.turn + (size_t)it.bh * p.nq + i;
+            if (ok && p.deterministic && h == 0) {
+              ok = wait_turn(turn, add_rank(p, it.j, i), w);
+              fence_proxy_async_global();
+            }
             if (ok) {
               bulk_reduce_add_f32(dst + h * GROUPS * 512, slot, C::DQ_PART_BYTES);
               bulk_commit_group();
               bulk_issued = true;
               bulk_wait_read_all();
+              if (p.deterministic && h + 1 == C::DQ_PARTS) {
+                // the additions are complete in global memory before the turn passes
+                bulk_wait_all();
+                fence_proxy_async_global();
+                red_release_add_gpu(turn, 1u);
+              }
               if (h + 1 < C::DQ_PARTS) {
                 mbar_arrive(&dq_half);
               } else {
@@ -805,6 +870,7 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
   float* Dw = reinterpret_cast<float*>(ws + wl.d_off);
   float* L2w = reinterpret_cast<float*>(ws + wl.l2_off);
   uint32_t* sched = reinterpret_cast<uint32_t*>(ws + wl.sched_off);
+  uint32_t* turn = reinterpret_cast<uint32_t*>(ws + wl.turn_off);
   const int sms = num_sms();
 
   if (stage < 0 || stage == 0) {
@@ -814,7 +880,7 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
     bwd::prep_kernel<D><<<(int)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(O),
                                                      static_cast<const __nv_bfloat16*>(dO), LSE, Dw, L2w, dq_acc,
-                                                     sched, pr.BH, pr.N, Npad);
+                                                     sched, turn, pr.BH, pr.N, Npad);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stage < 0 || stage == 1) {
@@ -835,6 +901,8 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     p.L2w = L2w;
     p.dq_acc = dq_acc;
     p.sched = sched;
+    p.turn = turn;
+    p.deterministic = pr.deterministic;
     p.group = pr.BH < 8 ? pr.BH : 8;
     p.dK = static_cast<__nv_bfloat16*>(dK);
     p.dV = static_cast<__nv_bfloat16*>(dV);

@@ -18,6 +18,7 @@ struct Problem {
   int off;         // Nk - N: causal alignment (query i sees keys j <= i + off)
   int mask_kind;
   const uint8_t* block_mask;  // device [nq, nk] or nullptr
+  int deterministic = 0;      // backward: fixed order of the dQ additions
   float scale;
   float scale_log2;  // scale * log2(e), computed in double and rounded once
 };

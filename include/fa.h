@@ -122,6 +122,23 @@ fa_status fa_fwd_qk(const void* Q, const void* K, const void* V, int B, int H, i
                     int mask_kind, const uint8_t* block_mask, float scale, void* O, float* LSE,
                     void* stream);
 size_t fa_bwd_workspace_size_qk(int B, int H, int Nq, int Nk, int d);
+
+/* fa_bwd_qk with run-to-run reproducible gradients: every element of dQ is
+ * summed over key tiles in ascending key-tile order (each key tile waits
+ * for its turn per query tile, through counters in the workspace), so the
+ * result is the same bits on every run with the same inputs on the same
+ * GPU.  dK and dV are always reproducible.  Same arguments, workspace size
+ * and errors as fa_bwd_qk; slower, since the dQ additions of a query tile
+ * are serialised.  It waits on other CTAs of the same launch: run it where
+ * the launch can occupy the GPU (a launch whose CTAs cannot all become
+ * resident within the wait limit ends with FA_ERR_TIMEOUT from
+ * fa_device_status()).  No page counterpart: the pages do not address
+ * reproducibility. */
+fa_status fa_bwd_qk_deterministic(const void* Q, const void* K, const void* V, const void* O,
+                                  const void* dO, const float* LSE, int B, int H, int Nq, int Nk,
+                                  int d, int mask_kind, const uint8_t* block_mask, float scale,
+                                  void* dQ, void* dK, void* dV, void* workspace,
+                                  size_t workspace_bytes, void* stream);
 fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                     const float* LSE, int B, int H, int Nq, int Nk, int d, int mask_kind,
                     const uint8_t* block_mask, float scale, void* dQ, void* dK, void* dV,

@@ -135,3 +135,46 @@ def test_bwd_workloads_every_head(name):
     assert (np.abs(dk.sum(axis=1)).max(axis=1) <= 2e-2 * kscale + 1e-6).all()
     vscale = np.abs(do).sum(axis=1).max(axis=1)
     assert (np.abs(dv.sum(axis=1) - do.sum(axis=1)).max(axis=1) <= 2e-2 * vscale).all()
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 1000, 128, "causal"), (2, 2, 640, 64, "none"),
+                                   (1, 2, 900, 64, "block"), (1, 2, 300, 700, 128, "causal")],
+                         ids=["1x2x1000x128-causal", "2x2x640x64-none", "1x2x900x64-block", "cross-300x700-causal"])
+def test_bwd_deterministic_reproducible_and_exact(shape):
+    """fa_bwd_qk_deterministic: the same bits on every run, and the oracle's
+    gradients within the usual tolerance."""
+    if len(shape) == 5:
+        B, H, N, d, m = shape
+        x = workloads.make_inputs(workloads.Workload("t", B, H, N, d, m, float(np.float32(d ** -0.5))), 8)
+    else:
+        B, H, N, Nk, d, m = shape
+        x = workloads.make_cross_inputs(B, H, N, Nk, d, m, seed=8)
+    scale = float(np.float32(d ** -0.5))
+    dv = to_dev(x)
+    O, L = fa.fwd(dv["Q"], dv["K"], dv["V"], m, dv["mask"], scale)
+    runs = [fa.bwd(dv["Q"], dv["K"], dv["V"], O, dv["dO"], L, m, dv["mask"], scale, deterministic=True)
+            for _ in range(3)]
+    assert fa.device_status() == 0
+    for r in runs[1:]:
+        for a, b in zip(runs[0], r):
+            assert torch.equal(a, b)
+    ref = oracle.bwd(x["Q"], x["K"], x["V"], x["dO"], m, x["mask"], scale)
+    for name, g in zip(("dQ", "dK", "dV"), runs[0]):
+        assert_grad(f64(g), ref[name], name, str(shape))
+
+
+@pytest.mark.parametrize("name", ["gpt2_s1k_causal", "long_s8k_d128_causal"])
+def test_bwd_deterministic_full_size(name):
+    """Full-size workloads: the ordered dQ additions complete (no wait runs
+    out), repeat bit for bit, and agree with the unordered backward."""
+    w = workloads.WORKLOADS[name]
+    dv = to_dev(workloads.make_inputs(w, 0))
+    O, L = fa.fwd(dv["Q"], dv["K"], dv["V"], w.mask, dv["mask"], w.scale)
+    a = fa.bwd(dv["Q"], dv["K"], dv["V"], O, dv["dO"], L, w.mask, dv["mask"], w.scale, deterministic=True)
+    b = fa.bwd(dv["Q"], dv["K"], dv["V"], O, dv["dO"], L, w.mask, dv["mask"], w.scale, deterministic=True)
+    c = fa.bwd(dv["Q"], dv["K"], dv["V"], O, dv["dO"], L, w.mask, dv["mask"], w.scale)
+    assert fa.device_status() == 0
+    for x, y, z in zip(a, b, c):
+        assert torch.equal(x, y)
+        err = (x.float() - z.float()).norm() / z.float().norm()
+        assert err.item() <= 1e-3
