@@ -41,6 +41,9 @@ SIGNATURES = {
                        _vp]),
     "fa_bwd_qk_deterministic": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp,
                                      _vp, _vp, _sz, _vp]),
+    "fa_fwd_varlen": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _vp, _vp, _vp]),
+    "fa_bwd_varlen": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _vp, _i, _vp, _vp,
+                           _vp, _vp, _sz, _vp]),
     "fa_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "fa_decode": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _sz, _vp]),
     "fa_standard_fwd_workspace_size": (_sz, [_i, _i, _i, _i]),
@@ -114,7 +117,17 @@ def _nk(Q, K, V):
     return K.shape[2]
 
 
-def fwd(Q, K, V, mask="none", block_mask=None, scale=None, O=None, LSE=None, stream=None):
+def _lens(t, B):
+    """Device pointer of an optional per-batch-element length vector."""
+    if t is None:
+        return None
+    if not (t.is_cuda and t.dtype == torch.int32 and t.is_contiguous() and t.numel() == B):
+        raise FAError(1, "sequence lengths must be a contiguous int32 CUDA tensor [B]")
+    return t.data_ptr()
+
+
+def fwd(Q, K, V, mask="none", block_mask=None, scale=None, O=None, LSE=None, stream=None, seqlens_q=None,
+        seqlens_k=None):
     """O [B,H,Nq,d] bf16 and LSE [B,H,Nq] fp32 (natural log); K, V are
     [B,H,Nk,d] (Nk may differ from Nq: fa_fwd_qk)."""
     _check_qkv(Q, K, V)
@@ -126,7 +139,11 @@ def fwd(Q, K, V, mask="none", block_mask=None, scale=None, O=None, LSE=None, str
         O = torch.empty_like(Q)
     if LSE is None:
         LSE = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
-    if Nk == N:
+    if seqlens_q is not None or seqlens_k is not None:
+        _check(lib().fa_fwd_varlen(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, H, N, Nk, d, kind, mptr, scale,
+                                   _lens(seqlens_q, B), _lens(seqlens_k, B), O.data_ptr(), LSE.data_ptr(),
+                                   _stream(stream)), "fa_fwd_varlen")
+    elif Nk == N:
         _check(lib().fa_fwd(Q.data_ptr(), K.data_ptr(), V.data_ptr(), B, H, N, d, kind, mptr, scale,
                             O.data_ptr(), LSE.data_ptr(), _stream(stream)), "fa_fwd")
     else:
@@ -142,7 +159,7 @@ def bwd_workspace_size(B, H, N, d, Nk=None) -> int:
 
 
 def bwd(Q, K, V, O, dO, LSE, mask="none", block_mask=None, scale=None, dQ=None, dK=None, dV=None,
-        workspace=None, stream=None, deterministic=False):
+        workspace=None, stream=None, deterministic=False, seqlens_q=None, seqlens_k=None):
     """dQ [B,H,Nq,d], dK, dV [B,H,Nk,d] bf16 (Nk may differ from Nq: fa_bwd_qk)."""
     _check_qkv(Q, K, V, O, dO)
     B, H, N, d = Q.shape
@@ -155,7 +172,13 @@ def bwd(Q, K, V, O, dO, LSE, mask="none", block_mask=None, scale=None, dQ=None, 
     ws = bwd_workspace_size(B, H, N, d, Nk)
     if workspace is None:
         workspace = torch.empty(ws, dtype=torch.uint8, device=Q.device)
-    if deterministic:
+    if seqlens_q is not None or seqlens_k is not None:
+        _check(lib().fa_bwd_varlen(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(), dO.data_ptr(),
+                                   LSE.data_ptr(), B, H, N, Nk, d, kind, mptr, scale, _lens(seqlens_q, B),
+                                   _lens(seqlens_k, B), 1 if deterministic else 0, dQ.data_ptr(), dK.data_ptr(),
+                                   dV.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)),
+               "fa_bwd_varlen")
+    elif deterministic:
         _check(lib().fa_bwd_qk_deterministic(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(), dO.data_ptr(),
                                              LSE.data_ptr(), B, H, N, Nk, d, kind, mptr, scale, dQ.data_ptr(),
                                              dK.data_ptr(), dV.data_ptr(), workspace.data_ptr(), workspace.numel(),

@@ -118,6 +118,19 @@ fa_status fa_fwd_qk(const void* Q, const void* K, const void* V, int B, int H, i
   return launch_fwd(p, Q, K, V, O, LSE, (cudaStream_t)stream);
 }
 
+fa_status fa_fwd_varlen(const void* Q, const void* K, const void* V, int B, int H, int Nq, int Nk, int d,
+                        int mask_kind, const uint8_t* block_mask, float scale, const int* seqlens_q,
+                        const int* seqlens_k, void* O, float* LSE, void* stream) {
+  if (!aligned(seqlens_q, 4) || !aligned(seqlens_k, 4)) return FA_ERR_INVALID_ARG;
+  Problem p;
+  fa_status st = check_common(Q, K, V, B, H, Nq, Nk, d, mask_kind, block_mask, scale, &p);
+  if (st != FA_OK) return st;
+  if (!O || !LSE || !aligned(O, 16) || !aligned(LSE, 4)) return FA_ERR_INVALID_ARG;
+  p.seqlens_q = seqlens_q;
+  p.seqlens_k = seqlens_k;
+  return launch_fwd(p, Q, K, V, O, LSE, (cudaStream_t)stream);
+}
+
 fa_status fa_fwd(const void* Q, const void* K, const void* V, int B, int H, int N, int d, int mask_kind,
                  const uint8_t* block_mask, float scale, void* O, float* LSE, void* stream) {
   return fa_fwd_qk(Q, K, V, B, H, N, N, d, mask_kind, block_mask, scale, O, LSE, stream);
@@ -137,10 +150,13 @@ size_t fa_bwd_workspace_size_qk(int B, int H, int Nq, int Nk, int d) {
 static fa_status bwd_common(int stage, const void* Q, const void* K, const void* V, const void* O, const void* dO,
                             const float* LSE, int B, int H, int N, int Nk, int d, int mask_kind,
                             const uint8_t* block_mask, float scale, void* dQ, void* dK, void* dV, void* workspace,
-                            size_t workspace_bytes, void* stream, int deterministic = 0) {
+                            size_t workspace_bytes, void* stream, int deterministic = 0,
+                            const int* seqlens_q = nullptr, const int* seqlens_k = nullptr) {
   Problem p;
   fa_status st = check_common(Q, K, V, B, H, N, Nk, d, mask_kind, block_mask, scale, &p);
   p.deterministic = deterministic;
+  p.seqlens_q = seqlens_q;
+  p.seqlens_k = seqlens_k;
   if (st != FA_OK) return st;
   if (!O || !dO || !LSE || !dQ || !dK || !dV) return FA_ERR_INVALID_ARG;
   if (!aligned(O, 16) || !aligned(dO, 16) || !aligned(LSE, 4) || !aligned(dQ, 16) || !aligned(dK, 16) ||
@@ -163,6 +179,16 @@ fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, 
                     void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_common(-1, Q, K, V, O, dO, LSE, B, H, Nq, Nk, d, mask_kind, block_mask, scale, dQ, dK, dV, workspace,
                     workspace_bytes, stream);
+}
+
+fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                        const float* LSE, int B, int H, int Nq, int Nk, int d, int mask_kind,
+                        const uint8_t* block_mask, float scale, const int* seqlens_q, const int* seqlens_k,
+                        int deterministic, void* dQ, void* dK, void* dV, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!aligned(seqlens_q, 4) || !aligned(seqlens_k, 4)) return FA_ERR_INVALID_ARG;
+  return bwd_common(-1, Q, K, V, O, dO, LSE, B, H, Nq, Nk, d, mask_kind, block_mask, scale, dQ, dK, dV, workspace,
+                    workspace_bytes, stream, deterministic ? 1 : 0, seqlens_q, seqlens_k);
 }
 
 fa_status fa_bwd_qk_deterministic(const void* Q, const void* K, const void* V, const void* O, const void* dO,

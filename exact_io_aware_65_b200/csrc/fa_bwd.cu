@@ -82,7 +82,8 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restri
                                                    const float* __restrict__ LSE, float* __restrict__ Dw,
                                                    float* __restrict__ L2w, float* __restrict__ dq_acc,
                                                    uint32_t* __restrict__ sched, uint32_t* __restrict__ turn,
-                                                   int BH, int N, int Npad) {
+                                                   int BH, int N, int Npad, int H,
+                                                   const int* __restrict__ seqlens_q) {
   constexpr int LPR = D / 8;
   if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0u;
   constexpr int RPW = 32 / LPR;
@@ -94,7 +95,9 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restri
        r0 += warps * RPW) {
     const long long r = r0 + sub;
     const int bh = (int)(r / Npad), n = (int)(r % Npad);
-    const bool real = r < total && n < N;
+    // rows past the sequence's length (or the padded count) are padding: P = 0
+    const int Lq = seqlens_q && r < total ? min(max(__ldg(seqlens_q + bh / H), 0), N) : N;
+    const bool real = r < total && n < Lq;
     float acc = 0.0f;
     if (real) {
       const size_t e = ((size_t)bh * N + n) * D + li * 8;
@@ -220,6 +223,9 @@ struct Params {
   const float* Dw;
   const float* L2w;
   float* dq_acc;
+  int H;             // heads per batch element
+  const int* seqlens_q;  // optional per-batch-element lengths (device int [B])
+  const int* seqlens_k;
   uint32_t* sched;
   uint32_t* turn;     // [BH, nq] dQ addition counters (deterministic mode)
   int deterministic;  // add each query tile's dQ parts in key-tile order
@@ -232,6 +238,7 @@ struct Params {
 
 struct Item {
   int bh, j;
+  int Lq, Lk, off, nqb;  // this sequence's query rows and keys, causal offset, query tiles
 };
 
 // Work item idx -> (head, key tile).  Heads are taken in groups of
@@ -239,6 +246,7 @@ struct Item {
 // to a few heads and stay in L2; within a group low key tiles come first
 // (under a causal mask they meet the most query tiles and run longest).
 
+template <bool VARLEN>
 __device__ __forceinline__ Item item_at(const Params& p, int idx) {
   const int per_group = p.group * p.nk;
   const int g = idx / per_group, r = idx % per_group;
@@ -246,6 +254,18 @@ __device__ __forceinline__ Item item_at(const Params& p, int idx) {
   Item it;
   it.j = r / gsize;
   it.bh = g * p.group + r % gsize;
+  if (VARLEN) {
+    const int b = it.bh / p.H;
+    it.Lq = p.seqlens_q ? min(max(__ldg(p.seqlens_q + b), 0), p.N) : p.N;
+    it.Lk = p.seqlens_k ? min(max(__ldg(p.seqlens_k + b), 0), p.Nk) : p.Nk;
+    it.off = it.Lk - it.Lq;
+    it.nqb = (it.Lq + BQ - 1) / BQ;
+  } else {  // every sequence fills its slice: the launch's own sizes
+    it.Lq = p.N;
+    it.Lk = p.Nk;
+    it.off = p.off;
+    it.nqb = p.nq;
+  }
   return it;
 }
 
@@ -299,23 +319,27 @@ __device__ bool wait_turn(const uint32_t* a, uint32_t want, const WaitCtx& w) {
 constexpr int RING = 4;     // depth of the item ring the producer fills
 constexpr int CONSUMERS = 13;  // MMA warp + 8 softmax warps + 4 drain warps
 
-// Next query tile >= i that attends to key tile j (nq if none).  Causal:
-// the rows that see some key of tile j are those >= j * BK - off.
-__device__ __forceinline__ int next_q(const Params& p, int j, int i) {
+// Next query tile >= i of the sequence that attends to key tile j (p.nq if
+// none; a key tile past the sequence's keys has none).  Causal: the rows
+// that see some key of tile j are those >= j * BK - off.
+template <bool VARLEN>
+__device__ __forceinline__ int next_q(const Params& p, const Item& it, int i) {
+  const int j = it.j;
+  if (VARLEN && j * BK >= it.Lk) return p.nq;
   if (p.mask_kind == FA_MASK_CAUSAL) {
-    const int first = max(0, j * BK - p.off) / BQ;
-    return i < first ? min(first, p.nq) : i;
+    const int first = max(0, j * BK - it.off) / BQ;
+    if (i < first) i = first;
+  } else if (p.mask_kind == FA_MASK_BLOCK) {
+    for (; i < it.nqb; ++i)
+      if (__ldg(p.block_mask + (size_t)i * p.nk + j)) break;
   }
-  if (p.mask_kind == FA_MASK_BLOCK) {
-    for (; i < p.nq; ++i)
-      if (__ldg(p.block_mask + (size_t)i * p.nk + j)) return i;
-  }
-  return i;
+  return (!VARLEN || i < it.nqb) ? i : p.nq;
 }
 
 
 
-template <int D>
+// VARLEN: per-sequence lengths are read (else every sequence has N, Nk).
+template <int D, bool VARLEN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                 const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapdO,
@@ -435,7 +459,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         item_ring[slot] = idx;
         mbar_arrive(&item_full[slot]);
         if (idx >= p.n_items) break;
-        const Item it = item_at(p, idx);
+        const Item it = item_at<VARLEN>(p, idx);
         ok = mbar_wait(&kv_empty, (item_iter & 1) ^ 1, w);
         if (!ok) break;
         mbar_arrive_expect_tx(&kv_full, 2 * C::TILE_BYTES);
@@ -444,7 +468,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_3d(sK + c * C::CHUNK_BYTES, &mapK, &kv_full, c * 64, it.j * BK, it.bh);
           tma_load_3d(sV + c * C::CHUNK_BYTES, &mapV, &kv_full, c * 64, it.j * BK, it.bh);
         }
-        for (int i = next_q(p, it.j, 0); i < p.nq; i = next_q(p, it.j, i + 1)) {
+        for (int i = next_q<VARLEN>(p, it, 0); i < p.nq; i = next_q<VARLEN>(p, it, i + 1)) {
           const uint32_t st = qd_iter % C::NST;
           const uint32_t par = ((qd_iter / C::NST) & 1) ^ 1;
           uint8_t* q = sQD + st * 2 * C::TILE_BYTES;
@@ -528,10 +552,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int idx;
         ok = take_item(item_iter, idx);
         if (!ok || idx >= p.n_items) break;
-        const Item it = item_at(p, idx);
+        const Item it = item_at<VARLEN>(p, idx);
         ok = mbar_wait(&kv_full, item_iter & 1, w);
         if (!ok) break;
-        int i = next_q(p, it.j, 0);
+        int i = next_q<VARLEN>(p, it, 0);
         if (i < p.nq) {
           ok = mbar_wait(&q_full[qd_iter % C::NST], (qd_iter / C::NST) & 1, w);
           if (!ok) break;
@@ -542,7 +566,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!ok) break;
         }
         for (int n = 0; ok && i < p.nq; ++n) {
-          const int inext = next_q(p, it.j, i + 1);
+          const int inext = next_q<VARLEN>(p, it, i + 1);
           const uint32_t st = qd_iter % C::NST;         // stage of query tile i
           const uint32_t stn = (qd_iter + 1) % C::NST;  // stage of query tile inext
           const uint32_t aQ = aQD + st * 2 * C::TILE_BYTES;
@@ -616,10 +640,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int idx;
       ok = take_item_warp(k, idx);
       if (!ok || idx >= p.n_items) break;
-      const Item it = item_at(p, idx);
+      const Item it = item_at<VARLEN>(p, idx);
       const int key = it.j * BK + kr;
       bool any = false;
-      for (int i = next_q(p, it.j, 0); i < p.nq; i = next_q(p, it.j, i + 1)) {
+      for (int i = next_q<VARLEN>(p, it, 0); i < p.nq; i = next_q<VARLEN>(p, it, i + 1)) {
         ok = mbar_wait_warp(&s_full, s_cnt & 1, w);
         if (!ok) break;
         const uint32_t par = s_cnt & 1;
@@ -631,12 +655,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float* sD = sL + 128;
         // causal: query row q sees this key iff key <= q + off; some pair in
         // the tile is hidden iff its last key exceeds its first row's limit
-        const bool cmask = p.mask_kind == FA_MASK_CAUSAL && it.j * BK + BK - 1 > i * BQ + p.off;
+        const bool cmask = p.mask_kind == FA_MASK_CAUSAL && it.j * BK + BK - 1 > i * BQ + it.off;
         // element masks only where the causal boundary or a ragged last key
         // tile crosses the tile: column c of this thread is hidden iff
         // c < kq, kq folding both tests (a missing key hides every column)
-        const bool masked = cmask || (it.j + 1) * BK > p.Nk;
-        const int kq = key >= p.Nk ? INT_MAX : (cmask ? key - (i * BQ + hf * 64 + p.off) : INT_MIN);
+        const bool masked = cmask || (it.j + 1) * BK > it.Lk;
+        const int kq = key >= it.Lk ? INT_MAX : (cmask ? key - (i * BQ + hf * 64 + it.off) : INT_MIN);
         // ---- P^T = exp2(S^T * scale * log2e - LSE_i * log2e), kept packed
         // as bf16 pairs (the form the dV product reads) for the dS step too.
         uint32_t pk[32];
@@ -766,8 +790,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int idx;
       ok = take_item_warp(k, idx);
       if (!ok || idx >= p.n_items) break;
-      const Item it = item_at(p, idx);
-      for (int i = next_q(p, it.j, 0); i < p.nq; i = next_q(p, it.j, i + 1)) {
+      const Item it = item_at<VARLEN>(p, idx);
+      for (int i = next_q<VARLEN>(p, it, 0); i < p.nq; i = next_q<VARLEN>(p, it, i + 1)) {
         const uint32_t b = dq_iter % C::NDQ;
         const uint32_t st = dq_iter % C::NST;
         ok = mbar_wait_warp(&dq_full[b], (dq_iter / C::NDQ) & 1, w);
@@ -880,7 +904,7 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
     bwd::prep_kernel<D><<<(int)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(O),
                                                      static_cast<const __nv_bfloat16*>(dO), LSE, Dw, L2w, dq_acc,
-                                                     sched, turn, pr.BH, pr.N, Npad);
+                                                     sched, turn, pr.BH, pr.N, Npad, pr.H, pr.seqlens_q);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stage < 0 || stage == 1) {
@@ -892,6 +916,9 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     p.Nk = pr.Nk;
     p.nk = pr.nk;
     p.off = pr.off;
+    p.H = pr.H;
+    p.seqlens_q = pr.seqlens_q;
+    p.seqlens_k = pr.seqlens_k;
     p.n_items = pr.BH * pr.nk;
     p.mask_kind = pr.mask_kind;
     p.block_mask = pr.block_mask;
@@ -909,10 +936,14 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     p.timeout_ns = wait_timeout_ns();
     p.status = st;
     constexpr int smem = bwd::Cfg<D>::SMEM_BYTES;
-    if (cudaFuncSetAttribute(bwd::main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return FA_ERR_CUDA;
     const int grid = p.n_items < sms ? p.n_items : sms;
-    bwd::main_kernel<D><<<grid, bwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, mdO, p);
+    auto run = [&](auto kern) -> bool {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return false;
+      kern<<<grid, bwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, mdO, p);
+      return true;
+    };
+    const bool varlen = pr.seqlens_q || pr.seqlens_k;
+    if (!(varlen ? run(bwd::main_kernel<D, true>) : run(bwd::main_kernel<D, false>))) return FA_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stage < 0 || stage == 2) {

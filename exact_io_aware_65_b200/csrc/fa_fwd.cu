@@ -76,6 +76,11 @@ struct Cfg {
 struct Params {
   int BH, N, nq, n_pairs, n_items, mask_kind;  // N, nq: query rows and tiles
   int Nk, nk, off;  // key rows and tiles; causal: query i sees keys j <= i + off
+  int H;            // heads per batch element (a head's batch element is bh / H)
+  // Optional per-batch-element lengths (device int [B], nullptr: N and Nk):
+  // query rows and keys at or past them are padding.
+  const int* seqlens_q;
+  const int* seqlens_k;
   int group;  // heads per scheduling group
   const uint8_t* block_mask;
   float scale_log2;
@@ -89,6 +94,7 @@ struct Params {
 struct Item {
   int bh, q0, q1;
   bool has1;
+  int Lq, Lk, off, nkb;  // this sequence's query rows and keys, causal offset, key tiles
 };
 
 // Work item idx -> (head, pair of query tiles).  Heads are taken in groups
@@ -96,6 +102,7 @@ struct Item {
 // in L2; within a group later query tiles come first, so that under a causal
 // mask the longest items start earliest (and, claimed dynamically, the short
 // ones fill in at the end).
+template <bool VARLEN>
 __device__ __forceinline__ Item item_at(const Params& p, int idx) {
   Item it;
   const int per_group = p.group * p.n_pairs;
@@ -106,41 +113,62 @@ __device__ __forceinline__ Item item_at(const Params& p, int idx) {
   it.q0 = 2 * c;
   it.q1 = 2 * c + 1;
   it.has1 = it.q1 < p.nq;
+  if (VARLEN) {
+    const int b = it.bh / p.H;
+    it.Lq = p.seqlens_q ? min(max(__ldg(p.seqlens_q + b), 0), p.N) : p.N;
+    it.Lk = p.seqlens_k ? min(max(__ldg(p.seqlens_k + b), 0), p.Nk) : p.Nk;
+    it.off = it.Lk - it.Lq;
+    it.nkb = (it.Lk + BN - 1) / BN;
+  } else {  // every sequence fills its slice: the launch's own sizes
+    it.Lq = p.N;
+    it.Lk = p.Nk;
+    it.off = p.off;
+    it.nkb = p.nk;
+  }
   return it;
 }
 
 // Last key a query row of tile qt may see under the causal mask (the tile's
-// last real row, shifted by the alignment; negative: none).
-__device__ __forceinline__ int causal_last_key(const Params& p, int qt) {
-  return min(qt * BM + BM - 1, p.N - 1) + p.off;
+// last row of the sequence, shifted by the alignment; negative: none).
+__device__ __forceinline__ int causal_last_key(const Item& it, int qt) {
+  return min(qt * BM + BM - 1, it.Lq - 1) + it.off;
 }
 
-// Does query tile qt attend to key tile j?
-__device__ __forceinline__ bool member(const Params& p, int qt, int j) {
-  if (p.mask_kind == FA_MASK_CAUSAL) return j * BN <= causal_last_key(p, qt);
+// Does query tile qt attend to key tile j?  (With per-sequence lengths,
+// tiles past the sequence's query rows or keys attend to nothing; without,
+// every tile an item or a key loop reaches is inside.)
+template <bool VARLEN>
+__device__ __forceinline__ bool member(const Params& p, const Item& it, int qt, int j) {
+  if (VARLEN && (qt * BM >= it.Lq || j >= it.nkb)) return false;
+  if (p.mask_kind == FA_MASK_CAUSAL) return j * BN <= causal_last_key(it, qt);
   if (p.mask_kind == FA_MASK_BLOCK) return __ldg(p.block_mask + (size_t)qt * p.nk + j) != 0;
   return true;
 }
 
 // One past the last key tile either query tile of the item may need.
+template <bool VARLEN>
 __device__ __forceinline__ int kv_end(const Params& p, const Item& it) {
+  if (VARLEN && it.q0 * BM >= it.Lq) return 0;
   if (p.mask_kind == FA_MASK_CAUSAL) {
-    const int last = causal_last_key(p, it.has1 ? it.q1 : it.q0);
-    return last < 0 ? 0 : min(p.nk, last / BN + 1);
+    const int last = causal_last_key(it, (it.has1 && (!VARLEN || it.q1 * BM < it.Lq)) ? it.q1 : it.q0);
+    return last < 0 ? 0 : min(it.nkb, last / BN + 1);
   }
-  return p.nk;
+  return it.nkb;
 }
 
 // Next key tile >= j needed by either query tile of the item (kv_end if none).
+template <bool VARLEN>
 __device__ __forceinline__ int next_union(const Params& p, const Item& it, int j) {
-  const int e = kv_end(p, it);
+  const int e = kv_end<VARLEN>(p, it);
   if (p.mask_kind != FA_MASK_BLOCK) return j < e ? j : e;
   for (; j < e; ++j)
-    if (member(p, it.q0, j) || (it.has1 && member(p, it.q1, j))) return j;
+    if (member<VARLEN>(p, it, it.q0, j) || (it.has1 && member<VARLEN>(p, it, it.q1, j))) return j;
   return e;
 }
 
-template <int D>
+// VARLEN: per-sequence lengths are read (else every sequence has N, Nk and
+// the sizes stay compile-time-free of extra registers).
+template <int D, bool VARLEN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                const __grid_constant__ CUtensorMap mapV, const Params p) {
@@ -234,7 +262,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         item_ring[slot] = idx;
         mbar_arrive(&item_full[slot]);
         if (idx >= p.n_items) break;
-        const Item it = item_at(p, idx);
+        const Item it = item_at<VARLEN>(p, idx);
         ok = mbar_wait(&q_empty, (item_iter & 1) ^ 1, w);
         if (!ok) break;
         mbar_arrive_expect_tx(&q_full, C::TILE_BYTES * (it.has1 ? 2 : 1));
@@ -246,8 +274,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int c = 0; c < C::CHUNKS; ++c)
             tma_load_3d(sQ + C::TILE_BYTES + c * C::CHUNK_BYTES, &mapQ, &q_full, c * 64, it.q1 * BM, it.bh);
         }
-        const int e = kv_end(p, it);
-        for (int j = next_union(p, it, 0); ok && j < e; j = next_union(p, it, j + 1)) {
+        const int e = kv_end<VARLEN>(p, it);
+        for (int j = next_union<VARLEN>(p, it, 0); ok && j < e; j = next_union<VARLEN>(p, it, j + 1)) {
           for (int kv = 0; kv < 2; ++kv) {
             const uint32_t slot = kv_iter % C::NSLOT;
             ok = mbar_wait(&kv_empty[slot], ((kv_iter / C::NSLOT) & 1) ^ 1, w);
@@ -323,14 +351,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int idx;
         ok = take_item(item_iter, idx);
         if (!ok || idx >= p.n_items) break;
-        const Item it = item_at(p, idx);
+        const Item it = item_at<VARLEN>(p, idx);
         const int tiles = it.has1 ? 2 : 1;  // tiles [0, tiles) exist
         ok = mbar_wait(&q_full, item_iter & 1, w);
         if (!ok) break;
         tc_fence_after();
-        const int e = kv_end(p, it);
-        int j = next_union(p, it, 0);
-        int jn = j < e ? next_union(p, it, j + 1) : e;  // the key tile after j
+        const int e = kv_end<VARLEN>(p, it);
+        int j = next_union<VARLEN>(p, it, 0);
+        int jn = j < e ? next_union<VARLEN>(p, it, j + 1) : e;  // the key tile after j
         bool first_pv[2] = {true, true};
         // Q is read only by the QK^T products: it goes back to the producer
         // once the item's last one has been issued, so the next item's Q
@@ -342,7 +370,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!ok) break;
           tc_fence_after();
           for (int t = t_lo; t < t_hi && t < tiles; ++t)
-            if (member(p, t == 0 ? it.q0 : it.q1, j)) issue_s(t, ks);
+            if (member<VARLEN>(p, it, t == 0 ? it.q0 : it.q1, j)) issue_s(t, ks);
           tc_commit(&kv_empty[ks]);
           ++kv_iter;
           if (jn >= e) {
@@ -351,7 +379,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         while (ok && j < e) {
-          const int jnn = jn < e ? next_union(p, it, jn + 1) : e;
+          const int jnn = jn < e ? next_union<VARLEN>(p, it, jn + 1) : e;
           const uint32_t vs = kv_iter % C::NSLOT;
           const uint32_t ksn = (kv_iter + 1) % C::NSLOT;
           ok = mbar_wait(&kv_full[vs], (kv_iter / C::NSLOT) & 1, w);
@@ -360,7 +388,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
           for (int t = t_lo; t < t_hi && t < tiles && ok; ++t) {
             const int qt = t == 0 ? it.q0 : it.q1;
-            if (member(p, qt, j)) {
+            if (member<VARLEN>(p, it, qt, j)) {
               ok = mbar_wait(&p_full[t], p_cnt[t] & 1, w);
               if (!ok) break;
               ++p_cnt[t];
@@ -368,7 +396,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               issue_pv(t, vs, first_pv[t] ? 0u : 1u);
               first_pv[t] = false;
             }
-            if (jn < e && member(p, qt, jn)) issue_s(t, ksn);
+            if (jn < e && member<VARLEN>(p, it, qt, jn)) issue_s(t, ksn);
           }
           if (!ok) break;
           tc_commit(&kv_empty[vs]);
@@ -415,16 +443,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int idx;
       ok = take_item_warp(k, idx);
       if (!ok || idx >= p.n_items) break;
-      const Item it = item_at(p, idx);
+      const Item it = item_at<VARLEN>(p, idx);
       if (t == 1 && !it.has1) continue;
       const int qt = t == 0 ? it.q0 : it.q1;
       const int row = qt * BM + r;
       float m = -INFINITY;  // reference maximum, scaled log2 units
       float l = 0.0f;
       bool first = true;  // no PV has written this tile's O yet
-      const int e = kv_end(p, it);
-      for (int j = next_union(p, it, 0); j < e; j = next_union(p, it, j + 1)) {
-        if (!member(p, qt, j)) continue;
+      const int e = kv_end<VARLEN>(p, it);
+      for (int j = next_union<VARLEN>(p, it, 0); j < e; j = next_union<VARLEN>(p, it, j + 1)) {
+        if (!member<VARLEN>(p, it, qt, j)) continue;
         ok = mbar_wait_warp(&s_full[t], s_cnt & 1, w);
         if (!ok) break;
         ++s_cnt;
@@ -439,8 +467,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // valid columns [0, lim): keys that exist and, under the causal mask,
         // keys <= row + off
         const int key0 = j * BN;
-        int lim = min(BN, p.Nk - key0);
-        if (p.mask_kind == FA_MASK_CAUSAL) lim = max(0, min(lim, row + p.off + 1 - key0));
+        int lim = min(BN, it.Lk - key0);
+        if (p.mask_kind == FA_MASK_CAUSAL) lim = max(0, min(lim, row + it.off + 1 - key0));
         if (lim < BN) {
 #pragma unroll
           for (int c = 0; c < BN; ++c)
@@ -506,7 +534,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       ++o_cnt;
       tc_fence_after();
-      const bool live = l > 0.0f;  // false only for a row that sees no key
+      const bool live = l > 0.0f && row < it.Lq;  // false for a row that sees no key, or padding
       const float inv_l = live ? 1.0f / l : 0.0f;
       __nv_bfloat16* orow = p.O + ((size_t)it.bh * p.N + row) * D;
 #pragma unroll
@@ -555,6 +583,9 @@ fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void
   p.Nk = pr.Nk;
   p.nk = pr.nk;
   p.off = pr.off;
+  p.H = pr.H;
+  p.seqlens_q = pr.seqlens_q;
+  p.seqlens_k = pr.seqlens_k;
   p.n_pairs = (pr.nq + 1) / 2;
   p.n_items = p.n_pairs * pr.BH;
   p.group = pr.BH < 8 ? pr.BH : 8;
@@ -568,18 +599,20 @@ fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void
   static std::atomic<uint32_t> next_slot{0};
   p.slot = next_slot.fetch_add(1u, std::memory_order_relaxed) % fwd::SCHED_SLOTS;
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
-  if (pr.d == 64) {
-    constexpr int smem = fwd::Cfg<64>::SMEM_BYTES;
-    if (cudaFuncSetAttribute(fwd::fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return FA_ERR_CUDA;
-    fwd::fwd_kernel<64><<<grid, fwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, p);
-  } else {
-    constexpr int smem = fwd::Cfg<128>::SMEM_BYTES;
-    if (cudaFuncSetAttribute(fwd::fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return FA_ERR_CUDA;
-    fwd::fwd_kernel<128><<<grid, fwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, p);
-  }
+  auto run = [&](auto kern, int smem) -> bool {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return false;
+    kern<<<grid, fwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, p);
+    return true;
+  };
+  const bool varlen = pr.seqlens_q || pr.seqlens_k;
+  bool ok;
+  if (pr.d == 64)
+    ok = varlen ? run(fwd::fwd_kernel<64, true>, fwd::Cfg<64>::SMEM_BYTES)
+                : run(fwd::fwd_kernel<64, false>, fwd::Cfg<64>::SMEM_BYTES);
+  else
+    ok = varlen ? run(fwd::fwd_kernel<128, true>, fwd::Cfg<128>::SMEM_BYTES)
+                : run(fwd::fwd_kernel<128, false>, fwd::Cfg<128>::SMEM_BYTES);
+  if (!ok) return FA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -19,6 +19,9 @@ struct Problem {
   int mask_kind;
   const uint8_t* block_mask;  // device [nq, nk] or nullptr
   int deterministic = 0;      // backward: fixed order of the dQ additions
+  // Optional per-batch-element lengths (device int [B]; nullptr: N, Nk).
+  const int* seqlens_q = nullptr;
+  const int* seqlens_k = nullptr;
   float scale;
   float scale_log2;  // scale * log2(e), computed in double and rounded once
 };

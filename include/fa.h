@@ -123,6 +123,28 @@ fa_status fa_fwd_qk(const void* Q, const void* K, const void* V, int B, int H, i
                     void* stream);
 size_t fa_bwd_workspace_size_qk(int B, int H, int Nq, int Nk, int d);
 
+/* Variable-length batches in padded storage: batch element b holds
+ * seqlens_q[b] query rows and seqlens_k[b] keys at the start of its
+ * [Nq, d] / [Nk, d] slices; the rest of each slice is padding.  Each
+ * sequence is its own attention problem (causal aligned at the bottom right
+ * of that sequence: row i sees keys j <= i + seqlens_k[b] - seqlens_q[b]);
+ * padding is never read as a key or a query, tiles wholly in padding do no
+ * work, and padding rows of the outputs come out as O = 0, LSE = -inf and
+ * zero gradients.  seqlens_q, seqlens_k: DEVICE int [B] (either may be NULL:
+ * every sequence then has Nq, or Nk); values are clamped to [0, Nq] and
+ * [0, Nk].  Otherwise as fa_fwd_qk / fa_bwd_qk (fa_bwd_qk_deterministic when
+ * deterministic != 0), with the same workspace.  No page counterpart beyond
+ * the batching of independent problems. */
+fa_status fa_fwd_varlen(const void* Q, const void* K, const void* V, int B, int H, int Nq, int Nk,
+                        int d, int mask_kind, const uint8_t* block_mask, float scale,
+                        const int* seqlens_q, const int* seqlens_k, void* O, float* LSE,
+                        void* stream);
+fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                        const float* LSE, int B, int H, int Nq, int Nk, int d, int mask_kind,
+                        const uint8_t* block_mask, float scale, const int* seqlens_q,
+                        const int* seqlens_k, int deterministic, void* dQ, void* dK, void* dV,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* fa_bwd_qk with run-to-run reproducible gradients: every element of dQ is
  * summed over key tiles in ascending key-tile order (each key tile waits
  * for its turn per query tile, through counters in the workspace), so the
