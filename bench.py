@@ -511,7 +511,7 @@ def decode_main(args, name, c):
     flop = 4 * B * H * Nq * Nk * d
     roofline = {"bound": "hbm", "kernel": "decode (partial + merge)", "achieved": achieved,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                "peak_source": f"{peak_kind} HBM copy bandwidth", "traffic": None,
+                "peak_source": f"{peak_kind} HBM copy bandwidth", "traffic": traffic_for("decode", name),
                 "source": "exact_io_aware_65_b200/csrc/fa_decode.cu"}
 
     # end to end: the cache stays resident (it is a cache); each step brings
