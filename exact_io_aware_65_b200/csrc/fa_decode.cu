@@ -12,7 +12,7 @@
 //
 // Kernel 1 (partial): persistent CTAs of 128 threads take work units (head,
 // chunk of CH keys) round-robin.  The 64-key tiles of K and V are contiguous
-// in [B,H,Nk,d], so each arrives by one bulk copy into a ring of stages.  Per
+// in [B,H,Nk,d], so each arrives by one bulk copy into a two-stage ring.  Per
 // tile and query: scores s = (scale log2 e) q . k, the running maximum m and
 // sum l of the online softmax, and O_u += 2^(s - m) V.  A unit leaves its
 // unnormalised O_u with m_u and l_u in the workspace.
@@ -30,7 +30,8 @@ namespace dec {
 
 constexpr int THREADS = 128;
 constexpr int TK = 64;      // keys per tile
-constexpr int NS = 3;       // ring stages
+constexpr int NS = 2;       // ring stages (small, so that three CTAs fit per SM at d = 128:
+                            // the per-tile block barriers are hidden by the other CTAs)
 constexpr int NQ_MAX = 16;  // query rows per head
 constexpr float LN2 = 0.69314718055994530942f;
 
@@ -77,7 +78,7 @@ __device__ __forceinline__ Unit unit_at(const Params& p, int u) {
 }
 
 template <int D, int NQT>
-__global__ void __launch_bounds__(THREADS, 2) partial_kernel(const Params p) {
+__global__ void __launch_bounds__(THREADS, 3) partial_kernel(const Params p) {
   using C = Cfg<D>;
   constexpr int QPT = qpt<D, NQT>();
   extern __shared__ __align__(128) uint8_t smem[];
