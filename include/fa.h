@@ -84,7 +84,8 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *      fa_bwd_workspace_size() bytes, contents irrelevant on entry).
  * Out: dQ, dK, dV [B,H,N,d] bf16, gradients of sum(dO * O) with respect to
  *      Q, K and V.  dQ is summed over key tiles in fp32 in an unspecified
- *      order, so its last bits may differ from run to run. */
+ *      order, so its last bits may differ from run to run
+ *      (fa_bwd_qk_deterministic fixes the order). */
 fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                  const float* LSE, int B, int H, int N, int d, int mask_kind,
                  const uint8_t* block_mask, float scale, void* dQ, void* dK, void* dV,
