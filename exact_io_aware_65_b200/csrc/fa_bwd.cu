@@ -133,32 +133,39 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restri
 }
 
 // --------------------------------------------------------------- convert ---
-// Thread g handles 8 columns of one query row; consecutive threads take
-// consecutive rows so the reads of the tiled accumulator are contiguous.
+// One CTA per (head, 128-row query tile): the tile is read in the
+// accumulator's own (tiled, contiguous) order into shared memory laid out by
+// rows (padded by 4 floats so successive rows start 4 banks apart), then
+// written out row by row: both global passes are contiguous.
 template <int D>
 __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict__ dq_acc,
                                                          __nv_bfloat16* __restrict__ dQ, int BH, int N, int Npad,
                                                          float scale) {
-  constexpr int PER_TILE = 128 * (D / 8);
+  constexpr int LD = D + 4;  // padded row length in shared memory (floats)
+  extern __shared__ __align__(16) float srow[];  // [128][LD]
   const int nq = Npad / 128;
-  const long long total = (long long)BH * nq * PER_TILE;
-  for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < total;
-       g += (long long)gridDim.x * blockDim.x) {
-    const long long tile = g / PER_TILE;  // bh * nq + qt
-    const int rem = (int)(g % PER_TILE);
-    const int e2 = rem / 128, r = rem % 128;
-    const int bh = (int)(tile / nq), qt = (int)(tile % nq);
+  const long long tile = blockIdx.x;  // bh * nq + qt
+  const int bh = (int)(tile / nq), qt = (int)(tile % nq);
+  const float* t = dq_acc + (size_t)tile * 128 * D;
+  // float4 f of the tile: column group e = f / 128, row r = f % 128
+  for (int f = threadIdx.x; f < 128 * D / 4; f += blockDim.x) {
+    const int e = f >> 7, r = f & 127;
+    *reinterpret_cast<float4*>(srow + r * LD + 4 * e) = reinterpret_cast<const float4*>(t)[f];
+  }
+  __syncthreads();
+  // 8 columns per thread; D/8 consecutive threads cover one output row
+  for (int g = threadIdx.x; g < 128 * (D / 8); g += blockDim.x) {
+    const int r = g / (D / 8), c = 8 * (g % (D / 8));
     const int n = qt * 128 + r;
     if (n >= N) continue;
-    const float* t = dq_acc + (size_t)tile * 128 * D;
-    const float4 a = *reinterpret_cast<const float4*>(t + (2 * e2) * 512 + r * 4);
-    const float4 b = *reinterpret_cast<const float4*>(t + (2 * e2 + 1) * 512 + r * 4);
+    const float4 a = *reinterpret_cast<const float4*>(srow + r * LD + c);
+    const float4 b = *reinterpret_cast<const float4*>(srow + r * LD + c + 4);
     uint4 o;
     o.x = pack_bf16x2(a.x * scale, a.y * scale);
     o.y = pack_bf16x2(a.z * scale, a.w * scale);
     o.z = pack_bf16x2(b.x * scale, b.y * scale);
     o.w = pack_bf16x2(b.z * scale, b.w * scale);
-    *reinterpret_cast<uint4*>(dQ + ((size_t)bh * N + n) * D + 8 * e2) = o;
+    *reinterpret_cast<uint4*>(dQ + ((size_t)bh * N + n) * D + c) = o;
   }
 }
 
@@ -947,11 +954,14 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stage < 0 || stage == 2) {
-    const long long work = (long long)pr.BH * Npad * (D / 8);
-    long long blocks = (work + 255) / 256;
-    if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
-    bwd::dq_convert_kernel<D><<<(int)blocks, 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), pr.BH, pr.N,
-                                                          Npad, pr.scale);
+    const long long tiles = (long long)pr.BH * (Npad / 128);
+    constexpr int smem = 128 * (D + 4) * (int)sizeof(float);
+    if (tiles > 0x7fffffffll ||
+        cudaFuncSetAttribute(bwd::dq_convert_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+      return FA_ERR_CUDA;
+    bwd::dq_convert_kernel<D><<<(unsigned)tiles, 256, smem, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), pr.BH,
+                                                                 pr.N, Npad, pr.scale);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;
