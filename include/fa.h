@@ -36,6 +36,11 @@
  *   - Ownership: the caller allocates and owns every buffer and the stream;
  *     the library keeps no allocation between calls.
  *   - Outputs must not alias inputs.
+ *   - CUDA graphs: every call can be captured into a graph, after one
+ *     eager call on the device has set up the per-device state.  Each
+ *     forward launch takes one of 4096 per-device work-counter slots when it
+ *     is issued, and a captured launch keeps its slot, so one graph must not
+ *     be replayed on two streams at once.
  *   - Errors: argument problems are reported synchronously, before anything
  *     is launched.  A failed launch returns FA_ERR_CUDA.  Every wait inside
  *     the kernels is bounded in time; a wait that runs out records
