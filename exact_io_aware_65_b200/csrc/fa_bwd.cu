@@ -133,39 +133,38 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restri
 }
 
 // --------------------------------------------------------------- convert ---
-// One CTA per (head, 128-row query tile): the tile is read in the
-// accumulator's own (tiled, contiguous) order into shared memory laid out by
-// rows (padded by 4 floats so successive rows start 4 banks apart), then
-// written out row by row: both global passes are contiguous.
+// Each thread takes 16 columns of one query row: four float4 column groups
+// of the tiled accumulator.  Consecutive threads take consecutive rows, so
+// every load instruction reads 512 contiguous bytes per warp, and each thread
+// writes one whole 32-byte sector of the bf16 row.
 template <int D>
 __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict__ dq_acc,
                                                          __nv_bfloat16* __restrict__ dQ, int BH, int N, int Npad,
                                                          float scale) {
-  constexpr int LD = D + 4;  // padded row length in shared memory (floats)
-  extern __shared__ __align__(16) float srow[];  // [128][LD]
+  constexpr int G = 4;                         // column groups per thread
+  constexpr int PER_TILE = 128 * (D / (4 * G));
   const int nq = Npad / 128;
-  const long long tile = blockIdx.x;  // bh * nq + qt
-  const int bh = (int)(tile / nq), qt = (int)(tile % nq);
-  const float* t = dq_acc + (size_t)tile * 128 * D;
-  // float4 f of the tile: column group e = f / 128, row r = f % 128
-  for (int f = threadIdx.x; f < 128 * D / 4; f += blockDim.x) {
-    const int e = f >> 7, r = f & 127;
-    *reinterpret_cast<float4*>(srow + r * LD + 4 * e) = reinterpret_cast<const float4*>(t)[f];
-  }
-  __syncthreads();
-  // 8 columns per thread; D/8 consecutive threads cover one output row
-  for (int g = threadIdx.x; g < 128 * (D / 8); g += blockDim.x) {
-    const int r = g / (D / 8), c = 8 * (g % (D / 8));
+  const long long total = (long long)BH * nq * PER_TILE;
+  for (long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x; g < total;
+       g += (long long)gridDim.x * blockDim.x) {
+    const long long tile = g / PER_TILE;  // bh * nq + qt
+    const int rem = (int)(g % PER_TILE);
+    const int eb = rem / 128, r = rem % 128;
+    const int bh = (int)(tile / nq), qt = (int)(tile % nq);
     const int n = qt * 128 + r;
+    // float4 f of a tile: column group f / 128, row f % 128
+    const float4* t = reinterpret_cast<const float4*>(dq_acc + (size_t)tile * 128 * D);
+    float4 v[G];
+#pragma unroll
+    for (int j = 0; j < G; ++j) v[j] = t[(eb * G + j) * 128 + r];
     if (n >= N) continue;
-    const float4 a = *reinterpret_cast<const float4*>(srow + r * LD + c);
-    const float4 b = *reinterpret_cast<const float4*>(srow + r * LD + c + 4);
-    uint4 o;
-    o.x = pack_bf16x2(a.x * scale, a.y * scale);
-    o.y = pack_bf16x2(a.z * scale, a.w * scale);
-    o.z = pack_bf16x2(b.x * scale, b.y * scale);
-    o.w = pack_bf16x2(b.z * scale, b.w * scale);
-    *reinterpret_cast<uint4*>(dQ + ((size_t)bh * N + n) * D + c) = o;
+    uint4* dst = reinterpret_cast<uint4*>(dQ + ((size_t)bh * N + n) * D + 4 * G * eb);
+#pragma unroll
+    for (int h = 0; h < G / 2; ++h) {
+      const float4 a = v[2 * h], b = v[2 * h + 1];
+      dst[h] = make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
+                          pack_bf16x2(b.x * scale, b.y * scale), pack_bf16x2(b.z * scale, b.w * scale));
+    }
   }
 }
 
@@ -954,14 +953,12 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stage < 0 || stage == 2) {
-    const long long tiles = (long long)pr.BH * (Npad / 128);
-    constexpr int smem = 128 * (D + 4) * (int)sizeof(float);
-    if (tiles > 0x7fffffffll ||
-        cudaFuncSetAttribute(bwd::dq_convert_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess)
-      return FA_ERR_CUDA;
-    bwd::dq_convert_kernel<D><<<(unsigned)tiles, 256, smem, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), pr.BH,
-                                                                 pr.N, Npad, pr.scale);
+    // one thread per 16 columns of a padded row; the loop covers any excess
+    const long long threads = (long long)pr.BH * Npad * (D / 16);
+    const long long blocks = (threads + 255) / 256;
+    const unsigned grid = (unsigned)(blocks < 0x7fffffffll ? blocks : 0x7fffffffll);
+    bwd::dq_convert_kernel<D><<<grid, 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), pr.BH, pr.N, Npad,
+                                                   pr.scale);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;
