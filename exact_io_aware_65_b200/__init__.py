@@ -21,11 +21,13 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libfa.so")
+# FA_LIBRARY selects another build of the same library, e.g. the
+# index-checking debug build libfa_debug.so.
+LIB_PATH = os.environ.get("FA_LIBRARY") or os.path.join(_HERE, "libfa.so")
 
 MASKS = {"none": 0, "causal": 1, "block": 2}
 STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
-          4: "FA_ERR_WORKSPACE", 5: "FA_ERR_TIMEOUT"}
+          4: "FA_ERR_WORKSPACE", 5: "FA_ERR_TIMEOUT", 6: "FA_ERR_BOUNDS"}
 
 # Every symbol include/fa.h declares, with its ctypes signature.
 _vp, _i, _f, _sz, _u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64

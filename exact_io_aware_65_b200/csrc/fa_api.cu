@@ -256,7 +256,8 @@ fa_status fa_device_status(void* stream) {
   if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return FA_ERR_CUDA;
   if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
   if (v == 0) return FA_OK;
-  return v == FA_DEV_ERR_TIMEOUT ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
+  if (v == FA_DEV_ERR_TIMEOUT) return FA_ERR_TIMEOUT;
+  return v == FA_DEV_ERR_BOUNDS ? FA_ERR_BOUNDS : FA_ERR_CUDA;
 }
 
 void fa_set_wait_timeout_ns(uint64_t ns) { g_wait_timeout_ns.store(ns ? ns : 4000000000ull); }
@@ -269,6 +270,7 @@ const char* fa_status_string(fa_status s) {
     case FA_ERR_CUDA: return "CUDA error";
     case FA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case FA_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+    case FA_ERR_BOUNDS: return "a device-side index check failed (debug build)";
   }
   return "unknown status";
 }

@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restri
                                                    float* __restrict__ L2w, float* __restrict__ dq_acc,
                                                    uint32_t* __restrict__ sched, uint32_t* __restrict__ turn,
                                                    int BH, int N, int Npad, int H,
-                                                   const int* __restrict__ seqlens_q) {
+                                                   const int* __restrict__ seqlens_q, uint32_t* status) {
   constexpr int LPR = D / 8;
   if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0u;
   constexpr int RPW = 32 / LPR;
@@ -96,10 +96,12 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restri
     const long long r = r0 + sub;
     const int bh = (int)(r / Npad), n = (int)(r % Npad);
     // rows past the sequence's length (or the padded count) are padding: P = 0
-    const int Lq = seqlens_q && r < total ? min(max(__ldg(seqlens_q + bh / H), 0), N) : N;
+    const int Lq = seqlens_q && r < total
+                       ? (FA_IN_BOUNDS(status, bh / H, 1, BH / H) ? min(max(__ldg(seqlens_q + bh / H), 0), N) : 0)
+                       : N;
     const bool real = r < total && n < Lq;
     float acc = 0.0f;
-    if (real) {
+    if (real && FA_IN_BOUNDS(status, ((size_t)bh * N + n) * D + li * 8, 8, (size_t)BH * N * D)) {
       const size_t e = ((size_t)bh * N + n) * D + li * 8;
       const uint4 a = *reinterpret_cast<const uint4*>(O + e);
       const uint4 b = *reinterpret_cast<const uint4*>(dO + e);
@@ -114,12 +116,13 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restri
     }
 #pragma unroll
     for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (r < total) {
+    if (r < total && FA_IN_BOUNDS(status, r, 1, total) && FA_IN_BOUNDS(status, r * D + li * 8, 8, total * D)) {
       if (li == 0) {
-        if ((n & 127) == 0) turn[(size_t)bh * (Npad / 128) + n / 128] = 0u;
+        if ((n & 127) == 0 && FA_IN_BOUNDS(status, (size_t)bh * (Npad / 128) + n / 128, 1, total / 128))
+          turn[(size_t)bh * (Npad / 128) + n / 128] = 0u;
         Dw[r] = acc;
         float l2 = INFINITY;  // padding rows and rows that saw no key: P = 0
-        if (real) {
+        if (real && FA_IN_BOUNDS(status, (size_t)bh * N + n, 1, (size_t)BH * N)) {
           const float lse = LSE[(size_t)bh * N + n];
           if (lse > -INFINITY) l2 = lse * LOG2E;
         }
@@ -140,7 +143,7 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restri
 template <int D>
 __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict__ dq_acc,
                                                          __nv_bfloat16* __restrict__ dQ, int BH, int N, int Npad,
-                                                         float scale) {
+                                                         float scale, uint32_t* status) {
   constexpr int G = 4;                         // column groups per thread
   constexpr int PER_TILE = 128 * (D / (4 * G));
   const int nq = Npad / 128;
@@ -156,8 +159,11 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict
     const float4* t = reinterpret_cast<const float4*>(dq_acc + (size_t)tile * 128 * D);
     float4 v[G];
 #pragma unroll
-    for (int j = 0; j < G; ++j) v[j] = t[(eb * G + j) * 128 + r];
-    if (n >= N) continue;
+    for (int j = 0; j < G; ++j)
+      v[j] = FA_IN_BOUNDS(status, tile * 128 * D + 4 * ((eb * G + j) * 128 + r), 4, total / PER_TILE * 128 * D)
+                 ? t[(eb * G + j) * 128 + r]
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (n >= N || !FA_IN_BOUNDS(status, ((size_t)bh * N + n) * D + 4 * G * eb, 4 * G, (size_t)BH * N * D)) continue;
     uint4* dst = reinterpret_cast<uint4*>(dQ + ((size_t)bh * N + n) * D + 4 * G * eb);
 #pragma unroll
     for (int h = 0; h < G / 2; ++h) {
@@ -262,8 +268,9 @@ __device__ __forceinline__ Item item_at(const Params& p, int idx) {
   it.bh = g * p.group + r % gsize;
   if (VARLEN) {
     const int b = it.bh / p.H;
-    it.Lq = p.seqlens_q ? min(max(__ldg(p.seqlens_q + b), 0), p.N) : p.N;
-    it.Lk = p.seqlens_k ? min(max(__ldg(p.seqlens_k + b), 0), p.Nk) : p.Nk;
+    const bool bok = FA_IN_BOUNDS(p.status, b, 1, p.BH / p.H);
+    it.Lq = p.seqlens_q ? (bok ? min(max(__ldg(p.seqlens_q + b), 0), p.N) : 0) : p.N;
+    it.Lk = p.seqlens_k ? (bok ? min(max(__ldg(p.seqlens_k + b), 0), p.Nk) : 0) : p.Nk;
     it.off = it.Lk - it.Lq;
     it.nqb = (it.Lq + BQ - 1) / BQ;
   } else {  // every sequence fills its slice: the launch's own sizes
@@ -282,7 +289,9 @@ __device__ __forceinline__ Item item_at(const Params& p, int idx) {
 __device__ __forceinline__ uint32_t add_rank(const Params& p, int j, int i) {
   if (p.mask_kind == FA_MASK_BLOCK) {
     uint32_t r = 0;
-    for (int k = 0; k < j; ++k) r += __ldg(p.block_mask + (size_t)i * p.nk + k) != 0;
+    for (int k = 0; k < j; ++k)
+      r += FA_IN_BOUNDS(p.status, (size_t)i * p.nk + k, 1, (size_t)p.nq * p.nk) &&
+           __ldg(p.block_mask + (size_t)i * p.nk + k) != 0;
     return r;
   }
   // no mask, or causal: a lower key tile is visible to every query row that
@@ -337,7 +346,9 @@ __device__ __forceinline__ int next_q(const Params& p, const Item& it, int i) {
     if (i < first) i = first;
   } else if (p.mask_kind == FA_MASK_BLOCK) {
     for (; i < it.nqb; ++i)
-      if (__ldg(p.block_mask + (size_t)i * p.nk + j)) break;
+      if (FA_IN_BOUNDS(p.status, (size_t)i * p.nk + j, 1, (size_t)p.nq * p.nk) &&
+          __ldg(p.block_mask + (size_t)i * p.nk + j))
+        break;
   }
   return (!VARLEN || i < it.nqb) ? i : p.nq;
 }
@@ -486,7 +497,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < C::CHUNKS; ++c)
             tma_load_3d(q + c * C::CHUNK_BYTES, &mapQ, &q_full[st], c * 64, i * BQ, it.bh);
-          bulk_load(ld, p.L2w + row0, 512, &q_full[st]);
+          // (a debug build that finds row0 out of range loads the first rows
+          // instead, so the barrier still gets its bytes)
+          bulk_load(ld, p.L2w + (FA_IN_BOUNDS(p.status, row0, 128, (size_t)p.BH * p.Npad) ? row0 : 0), 512,
+                    &q_full[st]);
           ok = mbar_wait(&do_empty[st], par, w);
           if (!ok) {
             ++qd_iter;
@@ -497,7 +511,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < C::CHUNKS; ++c)
             tma_load_3d(q + C::TILE_BYTES + c * C::CHUNK_BYTES, &mapdO, &do_full[st], c * 64, i * BQ, it.bh);
-          bulk_load(ld + 512, p.Dw + row0, 512, &do_full[st]);
+          bulk_load(ld + 512, p.Dw + (FA_IN_BOUNDS(p.status, row0, 128, (size_t)p.BH * p.Npad) ? row0 : 0), 512,
+                    &do_full[st]);
           ++qd_iter;
         }
         if (!ok) break;
@@ -770,7 +785,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             pk[e] = any ? pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul) : 0u;
-          if (store) {
+          if (store && FA_IN_BOUNDS(p.status, gbase + hf * (D / 2) + c, 32, (size_t)p.BH * p.Nk * D)) {
             uint4* o = reinterpret_cast<uint4*>(dst + hf * (D / 2) + c);
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
@@ -840,16 +855,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (leader) {
             ok = mbar_wait(&dq_staged[h], dq_iter & 1, w);
             uint32_t* turn = p.turn + (size_t)it.bh * p.nq + i;
-            if (ok && p.deterministic && h == 0) {
+            const bool turn_ok = !p.deterministic ||
+                                 FA_IN_BOUNDS(p.status, (size_t)it.bh * p.nq + i, 1, (size_t)p.BH * p.nq);
+            if (ok && p.deterministic && h == 0 && turn_ok) {
               ok = wait_turn(turn, add_rank(p, it.j, i), w);
               fence_proxy_async_global();
             }
             if (ok) {
-              bulk_reduce_add_f32(dst + h * GROUPS * 512, slot, C::DQ_PART_BYTES);
+              if (FA_IN_BOUNDS(p.status, ((size_t)it.bh * p.Npad + (size_t)i * BQ) * D + h * GROUPS * 512,
+                               C::DQ_PART_BYTES / 4, (size_t)p.BH * p.Npad * D))
+                bulk_reduce_add_f32(dst + h * GROUPS * 512, slot, C::DQ_PART_BYTES);
               bulk_commit_group();
               bulk_issued = true;
               bulk_wait_read_all();
-              if (p.deterministic && h + 1 == C::DQ_PARTS) {
+              if (p.deterministic && h + 1 == C::DQ_PARTS && turn_ok) {
                 // the additions are complete in global memory before the turn passes
                 bulk_wait_all();
                 fence_proxy_async_global();
@@ -910,7 +929,7 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
     bwd::prep_kernel<D><<<(int)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(O),
                                                      static_cast<const __nv_bfloat16*>(dO), LSE, Dw, L2w, dq_acc,
-                                                     sched, turn, pr.BH, pr.N, Npad, pr.H, pr.seqlens_q);
+                                                     sched, turn, pr.BH, pr.N, Npad, pr.H, pr.seqlens_q, st);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stage < 0 || stage == 1) {
@@ -958,7 +977,7 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     const long long blocks = (threads + 255) / 256;
     const unsigned grid = (unsigned)(blocks < 0x7fffffffll ? blocks : 0x7fffffffll);
     bwd::dq_convert_kernel<D><<<grid, 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), pr.BH, pr.N, Npad,
-                                                   pr.scale);
+                                                   pr.scale, st);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;

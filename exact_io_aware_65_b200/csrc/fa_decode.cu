@@ -108,7 +108,10 @@ __global__ void __launch_bounds__(THREADS, 3) partial_kernel(const Params p) {
     const uint32_t bytes = (uint32_t)rows * D * 2;
     const uint32_t s = issued % NS;
     uint8_t* kdst = smem + s * 2 * C::TILE_BYTES;
-    const size_t src = ((size_t)un.bh * p.Nk + k0) * D;
+    size_t src = ((size_t)un.bh * p.Nk + k0) * D;
+    // (a debug build that finds the tile out of range copies the cache's
+    // first rows instead, so the barrier still gets its bytes)
+    if (!FA_IN_BOUNDS(p.status, src, (size_t)rows * D, (size_t)p.BH * p.Nk * D)) src = 0;
     mbar_arrive_expect_tx(&full[s], 2 * bytes);
     bulk_load(kdst, p.K + src, bytes, &full[s]);
     bulk_load(kdst + C::TILE_BYTES, p.V + src, bytes, &full[s]);
@@ -127,7 +130,10 @@ __global__ void __launch_bounds__(THREADS, 3) partial_kernel(const Params p) {
     const Unit un = unit_at(p, u);
     // this head's queries (bf16, exact copies) and fresh softmax state
     for (int i = tid; i < p.Nq * D / 8; i += THREADS)
-      reinterpret_cast<uint4*>(sQ)[i] = reinterpret_cast<const uint4*>(p.Q + (size_t)un.bh * p.Nq * D)[i];
+      reinterpret_cast<uint4*>(sQ)[i] =
+          FA_IN_BOUNDS(p.status, (size_t)un.bh * p.Nq * D + 8 * i, 8, (size_t)p.BH * p.Nq * D)
+              ? reinterpret_cast<const uint4*>(p.Q + (size_t)un.bh * p.Nq * D)[i]
+              : make_uint4(0u, 0u, 0u, 0u);
     if (tid < NQ_MAX) {
       m_run[tid] = -INFINITY;
       l_run[tid] = 0.0f;
@@ -240,9 +246,11 @@ __global__ void __launch_bounds__(THREADS, 3) partial_kernel(const Params p) {
 #pragma unroll
       for (int qi = 0; qi < QPT; ++qi) {
         const int q = q0 + qi * qs;
-        if (q < p.Nq) p.part[((size_t)u * p.Nq + q) * D + c] = acc[qi];
+        if (q < p.Nq && FA_IN_BOUNDS(p.status, ((size_t)u * p.Nq + q) * D + c, 1, (size_t)p.n_units * p.Nq * D))
+          p.part[((size_t)u * p.Nq + q) * D + c] = acc[qi];
       }
-      if (tid < p.Nq) p.ml[(size_t)u * p.Nq + tid] = make_float2(m_run[tid], l_run[tid]);
+      if (tid < p.Nq && FA_IN_BOUNDS(p.status, (size_t)u * p.Nq + tid, 1, (size_t)p.n_units * p.Nq))
+        p.ml[(size_t)u * p.Nq + tid] = make_float2(m_run[tid], l_run[tid]);
     }
     __syncthreads();  // sQ and the softmax state are reused by the next unit
   }
@@ -257,6 +265,9 @@ template <int D>
 __global__ void __launch_bounds__(D) merge_kernel(const Params p, __nv_bfloat16* O, float* LSE) {
   const int bh = blockIdx.x / p.Nq, q = blockIdx.x % p.Nq, c = threadIdx.x;
   const int u0 = bh * p.nchunks;
+  if (!FA_IN_BOUNDS(p.status, ((size_t)bh * p.Nq + q) * D + c, 1, (size_t)p.BH * p.Nq * D) ||
+      !FA_IN_BOUNDS(p.status, (size_t)(u0 + p.nchunks - 1) * p.Nq + q, 1, (size_t)p.n_units * p.Nq))
+    return;
   float M = -INFINITY;
   for (int ch = 0; ch < p.nchunks; ++ch) M = fmaxf(M, p.ml[(size_t)(u0 + ch) * p.Nq + q].x);
   __nv_bfloat16* o = O + ((size_t)bh * p.Nq + q) * D;

@@ -115,8 +115,9 @@ __device__ __forceinline__ Item item_at(const Params& p, int idx) {
   it.has1 = it.q1 < p.nq;
   if (VARLEN) {
     const int b = it.bh / p.H;
-    it.Lq = p.seqlens_q ? min(max(__ldg(p.seqlens_q + b), 0), p.N) : p.N;
-    it.Lk = p.seqlens_k ? min(max(__ldg(p.seqlens_k + b), 0), p.Nk) : p.Nk;
+    const bool bok = FA_IN_BOUNDS(p.status, b, 1, p.BH / p.H);
+    it.Lq = p.seqlens_q ? (bok ? min(max(__ldg(p.seqlens_q + b), 0), p.N) : 0) : p.N;
+    it.Lk = p.seqlens_k ? (bok ? min(max(__ldg(p.seqlens_k + b), 0), p.Nk) : 0) : p.Nk;
     it.off = it.Lk - it.Lq;
     it.nkb = (it.Lk + BN - 1) / BN;
   } else {  // every sequence fills its slice: the launch's own sizes
@@ -141,7 +142,9 @@ template <bool VARLEN>
 __device__ __forceinline__ bool member(const Params& p, const Item& it, int qt, int j) {
   if (VARLEN && (qt * BM >= it.Lq || j >= it.nkb)) return false;
   if (p.mask_kind == FA_MASK_CAUSAL) return j * BN <= causal_last_key(it, qt);
-  if (p.mask_kind == FA_MASK_BLOCK) return __ldg(p.block_mask + (size_t)qt * p.nk + j) != 0;
+  if (p.mask_kind == FA_MASK_BLOCK)
+    return FA_IN_BOUNDS(p.status, (size_t)qt * p.nk + j, 1, (size_t)p.nq * p.nk) &&
+           __ldg(p.block_mask + (size_t)qt * p.nk + j) != 0;
   return true;
 }
 
@@ -546,13 +549,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           pk[i] = live ? pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l) : 0u;
-        if (row < p.N) {
+        if (row < p.N && FA_IN_BOUNDS(p.status, ((size_t)it.bh * p.N + row) * D + c, 32, (size_t)p.BH * p.N * D)) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
       }
-      if (row < p.N) p.LSE[(size_t)it.bh * p.N + row] = live ? (m + log2f(l)) * LN2 : -INFINITY;
+      if (row < p.N && FA_IN_BOUNDS(p.status, (size_t)it.bh * p.N + row, 1, (size_t)p.BH * p.N))
+        p.LSE[(size_t)it.bh * p.N + row] = live ? (m + log2f(l)) * LN2 : -INFINITY;
       tc_fence_before();
     }
   }

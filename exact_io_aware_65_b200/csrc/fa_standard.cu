@@ -32,18 +32,23 @@ constexpr float LN2 = 0.69314718055994530942f;
 __global__ void __launch_bounds__(THREADS) softmax_kernel(const float* __restrict__ S,
                                                           __nv_bfloat16* __restrict__ P, float* __restrict__ LSE,
                                                           int N, int mask_kind, const uint8_t* __restrict__ bm,
-                                                          int nb) {
+                                                          int nb, uint32_t* status) {
   extern __shared__ float row[];
   __shared__ float red[THREADS / 32];
   const size_t r = blockIdx.x;  // row index over B*H*N
   const int i = (int)(r % N);
   const float* s = S + r * N;
+  // the grid is one CTA per row of S, so every index below is in range; the
+  // debug build checks the row anyway
+  if (!FA_IN_BOUNDS(status, r * N, N, (size_t)gridDim.x * N)) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   float mx = -INFINITY;
   for (int j = tid; j < N; j += THREADS) {
     bool keep = true;
     if (mask_kind == FA_MASK_CAUSAL) keep = j <= i;
-    else if (mask_kind == FA_MASK_BLOCK) keep = bm[(size_t)(i / 128) * nb + j / 128] != 0;
+    else if (mask_kind == FA_MASK_BLOCK)
+      keep = FA_IN_BOUNDS(status, (size_t)(i / 128) * nb + j / 128, 1, (size_t)nb * nb) &&
+             bm[(size_t)(i / 128) * nb + j / 128] != 0;
     const float v = keep ? s[j] * LOG2E : -INFINITY;  // log2 units
     row[j] = v;
     mx = fmaxf(mx, v);
@@ -120,6 +125,8 @@ fa_status launch_standard_fwd(const Problem& pr, const void* Q, const void* K, c
   using namespace stdattn;
   cublasHandle_t h = blas_handle();
   if (!h) return FA_ERR_CUDA;
+  uint32_t* st = status_word();
+  if (!st) return FA_ERR_CUDA;
   const int N = pr.N, d = pr.d, BH = pr.BH;
   const size_t nn = (size_t)BH * N * N;
   float* S = static_cast<float*>(workspace);
@@ -138,7 +145,7 @@ fa_status launch_standard_fwd(const Problem& pr, const void* Q, const void* K, c
       cudaSuccess)
     return FA_ERR_CUDA;
   softmax_kernel<<<(unsigned)((size_t)BH * N), THREADS, (size_t)N * sizeof(float), s>>>(
-      S, P, LSE, N, pr.mask_kind, pr.block_mask, nb);
+      S, P, LSE, N, pr.mask_kind, pr.block_mask, nb, st);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   // O (row-major N x d) is stored as the column-major product V^T P^T:
   // A = V (stored d x N), B = P (stored N x N).

@@ -17,7 +17,26 @@ namespace fa {
 // Kernels report failures through a device status word (one per device,
 // module-scope in fa_api.cu; its address is passed to every launch).
 // 0 = ok; otherwise the first error code a kernel recorded.
-enum : uint32_t { FA_DEV_OK = 0, FA_DEV_ERR_TIMEOUT = 5 };
+enum : uint32_t { FA_DEV_OK = 0, FA_DEV_ERR_TIMEOUT = 5, FA_DEV_ERR_BOUNDS = 6 };
+
+// Index checks of the debug build (compiled with -DFA_DEBUG_BOUNDS).  Every
+// access a kernel makes through a raw global pointer names the elements it
+// touches, [first, first + count), and the buffer's extent in elements.
+// Accesses through a TMA tensor map need no check: the hardware clips the
+// box to the map.  In the debug build an access outside its buffer records
+// FA_DEV_ERR_BOUNDS in the status word and is skipped.  In the normal build
+// the check is the constant true and its arguments are never evaluated.
+#ifdef FA_DEBUG_BOUNDS
+__device__ __forceinline__ bool in_bounds(uint32_t* status, long long first, long long count, long long extent) {
+  if (first >= 0 && count >= 0 && first <= extent - count) return true;
+  atomicCAS(status, FA_DEV_OK, FA_DEV_ERR_BOUNDS);
+  return false;
+}
+#define FA_IN_BOUNDS(status, first, count, extent) \
+  ::fa::in_bounds((status), (long long)(first), (long long)(count), (long long)(extent))
+#else
+#define FA_IN_BOUNDS(status, first, count, extent) true
+#endif
 
 struct WaitCtx {
   uint64_t timeout_ns;       // how long one wait may last before it gives up

@@ -63,7 +63,9 @@ typedef enum {
   FA_ERR_UNSUPPORTED = 2, /* valid request outside this build: d not 64/128, sizes beyond int range */
   FA_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed */
   FA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than fa_bwd_workspace_size() */
-  FA_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out (see fa_device_status) */
+  FA_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out (see fa_device_status) */
+  FA_ERR_BOUNDS = 6       /* debug build only (libfa_debug.so): a kernel's index check
+                             found an access outside its buffer and skipped it */
 } fa_status;
 
 typedef enum { FA_MASK_NONE = 0, FA_MASK_CAUSAL = 1, FA_MASK_BLOCK = 2 } fa_mask_kind;
@@ -241,7 +243,8 @@ fa_status fa_bwd_static_workspace(const void* Q, const void* K, const void* V, c
 
 /* Synchronise `stream`, then read and clear the calling device's status
  * word.  Returns FA_OK, FA_ERR_TIMEOUT if a bounded wait ran out in a kernel
- * since the last call, or FA_ERR_CUDA if the synchronisation itself failed. */
+ * since the last call, FA_ERR_BOUNDS if (debug build only) an index check
+ * failed, or FA_ERR_CUDA if the synchronisation itself failed. */
 fa_status fa_device_status(void* stream);
 
 /* Set the wall-clock limit, in nanoseconds, of every device-side wait in

@@ -28,9 +28,27 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(L, name), name
 
 
+def test_debug_build_has_the_same_abi():
+    """The index-checking debug build (libfa_debug.so, built by
+    ``__graft_entry__.build()``) exports the same functions and rejects bad
+    arguments the same way."""
+    from exact_io_aware_65_b200 import build
+    if not os.path.exists(build.DEBUG_LIB):
+        pytest.skip("debug build not present (python -m exact_io_aware_65_b200.build --debug-bounds)")
+    L = ctypes.CDLL(build.DEBUG_LIB)
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    f = L.fa_status_string
+    f.restype, f.argtypes = ctypes.c_char_p, [ctypes.c_int]
+    assert f(6) and f(6) != fa.lib().fa_status_string(99)
+    g = L.fa_bwd_workspace_size
+    g.restype, g.argtypes = ctypes.c_size_t, [ctypes.c_int] * 4
+    assert g(2, 4, 4096, 128) == fa.bwd_workspace_size(2, 4, 4096, 128)
+
+
 def test_status_strings():
     L = fa.lib()
-    for code in range(6):
+    for code in range(7):
         assert L.fa_status_string(code)
     assert L.fa_status_string(0) == b"ok"
 
