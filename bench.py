@@ -178,8 +178,11 @@ def reference_arm(args, w):
         v, dt, desc, cores = cpu_sample(w, x, x["mask"], n)
         vals.append(v)
         secs += dt
-    value = (args.steps * (flops(w.with_(B=1, H=1, N=n), x["mask"])["fwd"] +
-                           flops(w.with_(B=1, H=1, N=n), x["mask"])["bwd"])) / secs / 1e12
+    # the work of one step: one head, the first n positions (and, for a block
+    # mask, the part of the tile grid those positions cover)
+    sub = w.with_(B=1, H=1, N=n)
+    f = flops(sub, x["mask"][: sub.nb, : sub.nb] if x["mask"] is not None else None)
+    value = args.steps * (f["fwd"] + f["bwd"]) / secs / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",

@@ -3,27 +3,32 @@ prints one JSON line with the same metric, unit and workload names as the
 CUDA arm, and under a multi-rank launch only rank 0 does any work."""
 import json
 import os
+import re
 import subprocess
 import sys
+
+import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
+import workloads  # noqa: E402
 
 
-def _run(extra_env=None, *args):
+def _run(extra_env=None, workload="tiny"):
     env = dict(os.environ)
     env.pop("RANK", None)
     env.pop("WORLD_SIZE", None)
     env.update(extra_env or {})
-    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
-           "--steps", "2", "--warmup", "3", *args]
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", workload,
+           "--steps", "2", "--warmup", "3"]
     return subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
 
 
-def test_reference_arm_prints_one_contract_line():
-    r = _run()
+@pytest.mark.parametrize("workload", list(workloads.WORKLOADS))
+def test_reference_arm_prints_one_contract_line(workload):
+    r = _run(workload=workload)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.strip()]
     assert len(lines) == 1, r.stdout
@@ -33,7 +38,11 @@ def test_reference_arm_prints_one_contract_line():
     assert d["higher_is_better"] is True and d["scaling"] == "weak" and d["vs_baseline"] is None
     assert d["n_gpus"] == 1 and d["steps"] == 2 and d["warmup"] == 3
     assert d["value"] > 0 and d["ms_per_step"] > 0
-    assert d["config"]["workload"] == "tiny"
+    assert d["config"]["workload"] == workload
+    # the value is the sampled work (14 d flops per kept score entry, fwd + bwd) over the step time
+    w = workloads.WORKLOADS[workload]
+    E = int(re.search(r"\((\d+) kept score entries per head\)", d["cpu_baseline"]["sample"]).group(1))
+    assert d["value"] == pytest.approx(14 * w.d * E / (d["ms_per_step"] * 1e-3) / 1e12, rel=1e-9)
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["unit"] == d["unit"]
     assert cb["cores"] >= 1 and cb["sample"]
