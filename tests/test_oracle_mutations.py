@@ -12,7 +12,10 @@ import oracle
 from oracle import build as obuild
 import test_oracle_pins as pins
 
-# (name, text in oracle.c, replacement, number of occurrences to replace)
+# (name, text in oracle.c, replacement).  A change that cannot alter any
+# result is left out.  Dropping pass 2's skip of rows whose LSE is -inf is
+# one: pass 2 only reaches a row through an allowed (row, key) pair, and such
+# a row always has a finite LSE.
 MUTANTS = [
     ("causal_off_by_one", "case OR_MASK_CAUSAL: return j <= i + (s->Nk - s->Nq);",
      "case OR_MASK_CAUSAL: return j < i + (s->Nk - s->Nq);"),
@@ -34,6 +37,18 @@ MUTANTS = [
     ("D_dropped_in_pass2", "double ds = p * (dp - Dv[(size_t)h * Nq + i]);", "double ds = p * dp;"),
     ("pv_wrong_row", "const double *v = V + hk + (size_t)j * d;\n                    for (int k = 0; k < d; ++k) o[k] += P[j] * v[k];\n                }\n            }\n        free(P);\n    }\n    return err;\n}\n\nint oracle_fwd(",
      "const double *v = V + hk + (size_t)(Nk - 1 - j) * d;\n                    for (int k = 0; k < d; ++k) o[k] += P[j] * v[k];\n                }\n            }\n        free(P);\n    }\n    return err;\n}\n\nint oracle_fwd("),
+    # a row that sees no key: the running maximum must start at -inf
+    ("empty_row_max_init", "double m = -INFINITY;", "double m = 0.0;"),
+    ("pass2_scale_dropped", "double p = exp(s.scale * dot(qi, kj, d) - L);", "double p = exp(dot(qi, kj, d) - L);"),
+    ("dK_scale_dropped", "for (int k = 0; k < d; ++k) dk[k] *= scale;", ""),
+    ("dV_wrong_operand", "dv[k] += p * doi[k];", "dv[k] += p * qi[k];"),
+    ("dQ_uses_V", "double ds = P[j] * (dP[j] - Di);\n                    const double *kj = K + hk",
+     "double ds = P[j] * (dP[j] - Di);\n                    const double *kj = V + hk"),
+    # the block grid's row length is the number of key blocks
+    ("block_row_length_from_queries", "s.nbk = (Nk + s.block - 1) / s.block;", "s.nbk = (Nq + s.block - 1) / s.block;"),
+    # the single-row path used for sampled parity at full size
+    ("rows_dS_sign", "double ds = P[j] * (dot(doi, V + hk + (size_t)j * d, d) - Di);",
+     "double ds = P[j] * (dot(doi, V + hk + (size_t)j * d, d) + Di);"),
 ]
 
 # The pins each mutant is run against (all cheap).
@@ -52,6 +67,7 @@ PIN_CALLS = [
     ("cross_suffix", lambda gd: pins.test_cross_causal_suffix_equals_square_problem()),
     ("cross_more_queries", lambda gd: pins.test_cross_causal_more_queries_than_keys()),
     ("cross_block", lambda gd: pins.test_cross_block_mask_is_query_blocks_by_key_blocks()),
+    ("rows_block", lambda gd: pins.test_row_path_matches_full_path("block")),
 ]
 
 
