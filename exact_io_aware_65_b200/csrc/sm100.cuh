@@ -27,9 +27,14 @@ enum : uint32_t { FA_DEV_OK = 0, FA_DEV_ERR_TIMEOUT = 5, FA_DEV_ERR_BOUNDS = 6 }
 // FA_DEV_ERR_BOUNDS in the status word and is skipped.  In the normal build
 // the check is the constant true and its arguments are never evaluated.
 #ifdef FA_DEBUG_BOUNDS
-__device__ __forceinline__ bool in_bounds(uint32_t* status, long long first, long long count, long long extent) {
+__host__ __device__ __forceinline__ bool in_bounds(uint32_t* status, long long first, long long count,
+                                                   long long extent) {
   if (first >= 0 && count >= 0 && first <= extent - count) return true;
+#ifdef __CUDA_ARCH__
   atomicCAS(status, FA_DEV_OK, FA_DEV_ERR_BOUNDS);
+#else
+  if (status && *status == FA_DEV_OK) *status = FA_DEV_ERR_BOUNDS;  // host callers (tests)
+#endif
   return false;
 }
 #define FA_IN_BOUNDS(status, first, count, extent) \
@@ -37,6 +42,17 @@ __device__ __forceinline__ bool in_bounds(uint32_t* status, long long first, lon
 #else
 #define FA_IN_BOUNDS(status, first, count, extent) true
 #endif
+
+// Read-only load: through the non-coherent read-only path on the device, a
+// plain load on the host (for host-callable schedule functions).
+template <typename T>
+__host__ __device__ __forceinline__ T ld_ro(const T* p) {
+#ifdef __CUDA_ARCH__
+  return __ldg(p);
+#else
+  return *p;
+#endif
+}
 
 struct WaitCtx {
   uint64_t timeout_ns;       // how long one wait may last before it gives up
