@@ -23,8 +23,9 @@
 //              P^T, dS^T                                   (softmax warps)
 //              dV  += P^T dO_i,   dK += dS^T Q_i            (A from tensor memory)
 //              dQ_i = dS K_j                                 (A = dS^T in smem)
-//            and dQ_i is added to the fp32 accumulator with vector
-//            reductions by four drain warps.
+//            Four drain warps read dQ_i out of tensor memory, stage it in a
+//            dead shared-memory buffer and add it to the fp32 accumulator
+//            with bulk reduce-adds (cp.reduce.async.bulk, add.f32).
 //   convert  dQ = bf16(scale * dQ_acc).
 //
 // CTA roles (512 threads): warp 0 TMA producer; warp 1 MMA issuer; warps

@@ -229,8 +229,16 @@ fa_status fa_standard_fwd(const void* Q, const void* K, const void* V, int B, in
  *     B*H*ceil(N/128)*128 up to about 129,000 for d = 128 and about 254,000
  *     for d = 64).
  *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture begins.
+ *     (cudaGetSymbolAddress, with that device current).  With the CUDA
+ *     runtime's lazy module loading (the default since CUDA 12.2) that first
+ *     call is also where the runtime reserves the 64 MiB on the device.  A
+ *     caller whose pool takes the device's memory should therefore make its
+ *     first call before the pool reserves that memory, and before any stream
+ *     capture begins.  Later calls allocate nothing.
+ *   - The looked-up address belongs to the device's context: after
+ *     cudaDeviceReset() on a device, this library must not be called on that
+ *     device again in the same process (this also holds for every other call
+ *     here, whose device status word is looked up the same way).
  *   - All calls on a device share the one array, and it keeps whatever the
  *     last call left in it (each call clears what must start at zero).  Calls
  *     whose kernels overlap on the GPU -- on different streams, or from

@@ -49,8 +49,11 @@ def load(path: str):
     L.oracle_rows_qk.argtypes = [_dp, _dp, _dp, _dp, i, i, i, i, i, _u8p, i, d,
                                  _ip, _ip, i, _dp, _dp, _dp]
     L.oracle_probs_qk.argtypes = [_dp, _dp, i, i, i, i, i, _u8p, i, d, _dp]
+    L.oracle_cols_qk.argtypes = [_dp, _dp, _dp, _dp, i, i, i, i, i, _u8p, i, d,
+                                 _ip, _ip, i, _dp, _dp]
     for f in (L.oracle_fwd, L.oracle_bwd, L.oracle_rows, L.oracle_probs,
-              L.oracle_fwd_qk, L.oracle_bwd_qk, L.oracle_rows_qk, L.oracle_probs_qk):
+              L.oracle_fwd_qk, L.oracle_bwd_qk, L.oracle_rows_qk, L.oracle_probs_qk,
+              L.oracle_cols_qk):
         f.restype = i
     return L
 
@@ -180,6 +183,26 @@ def rows(Q, K, V, heads, rws, dO=None, mask_kind="none", block_mask=None, scale=
                                 scale, hs.ctypes.data_as(_ip), rs.ctypes.data_as(_ip), R,
                                 _ptr(O), _ptr(L), _ptr(dQ)))
     return (O, L, dQ) if do is not None else (O, L)
+
+
+def cols(Q, K, V, dO, heads, keys, mask_kind="none", block_mask=None, scale=None, block=128):
+    """dK [C, d] and dV [C, d] for the key rows ``(heads[c], keys[c])``;
+    ``heads`` index the flattened B*H axis.  Costs one forward over the
+    heads named, plus O(Nq d) per key."""
+    q, k, v, do = _f64(Q), _f64(K), _f64(V), _f64(dO)
+    lead, BH, N, d = _shape(q)
+    Nk = _nk(k, BH, d)
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    kind, m, mp = _mask_args(block_mask, mask_kind)
+    hs = np.ascontiguousarray(np.asarray(heads, dtype=np.int32))
+    ks = np.ascontiguousarray(np.asarray(keys, dtype=np.int32))
+    C = len(hs)
+    dK = np.empty((C, d))
+    dV = np.empty((C, d))
+    _check(lib().oracle_cols_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(do), BH, N, Nk, d, kind, mp, block,
+                                scale, hs.ctypes.data_as(_ip), ks.ctypes.data_as(_ip), C,
+                                _ptr(dK), _ptr(dV)))
+    return dK, dV
 
 
 def probs(Q, K, mask_kind="none", block_mask=None, scale=None, block=128):

@@ -352,6 +352,93 @@ int oracle_rows(const double *Q, const double *K, const double *V, const double 
     return oracle_rows_qk(Q, K, V, dO, BH, N, N, d, kind, block_mask, block, scale, head, row, nrows, O, LSE, dQ);
 }
 
+/* Selected key columns: for each (head[c], col[c]) pair, dK_c [d] and
+ * dV_c [d], the gradients of one key row.  They sum over the query rows that
+ * see the key, and each such row enters through its normaliser LSE_i and its
+ * D_i = sum_j P_ij dP_ij, which depend on the whole score row.  So the row
+ * statistics of every head named in the list are computed first, row by row
+ * from the definition; then each requested column is a plain loop over the
+ * query rows:
+ *     P_ij = exp(scale q_i . k_j - LSE_i),  dP_ij = dO_i . v_j,
+ *     dS_ij = P_ij (dP_ij - D_i),
+ *     dV_j = sum_i P_ij dO_i,  dK_j = scale sum_i dS_ij q_i.
+ * The cost is one forward over the named heads plus O(Nq d) per column. */
+int oracle_cols_qk(const double *Q, const double *K, const double *V, const double *dO,
+                   int BH, int Nq, int Nk, int d, int kind, const uint8_t *block_mask, int block,
+                   double scale, const int *head, const int *col, int ncols,
+                   double *dK, double *dV)
+{
+    spec_t s = make_spec(Nq, Nk, d, kind, block_mask, block, scale);
+    if (check(&s, BH) != OR_OK || !Q || !K || !V || !dO || !head || !col || ncols < 0 || !dK || !dV)
+        return OR_ERR_ARG;
+    for (int c = 0; c < ncols; ++c)
+        if (head[c] < 0 || head[c] >= BH || col[c] < 0 || col[c] >= Nk) return OR_ERR_ARG;
+    unsigned char *need = (unsigned char *)calloc((size_t)BH, 1);
+    double *lse = (double *)malloc(sizeof(double) * (size_t)BH * Nq);
+    double *Dv = (double *)malloc(sizeof(double) * (size_t)BH * Nq);
+    if (!need || !lse || !Dv) { free(need); free(lse); free(Dv); return OR_ERR_NOMEM; }
+    for (int c = 0; c < ncols; ++c) need[head[c]] = 1;
+    int err = OR_OK;
+
+    /* row statistics of the named heads */
+#pragma omp parallel
+    {
+        double *P = (double *)malloc(sizeof(double) * (size_t)Nk);
+        if (!P) {
+#pragma omp atomic write
+            err = OR_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 8) collapse(2)
+        for (int h = 0; h < BH; ++h)
+            for (int i = 0; i < Nq; ++i) {
+                if (!P || !need[h]) continue;
+                const size_t hq = (size_t)h * Nq * d, hk = (size_t)h * Nk * d;
+                const double *doi = dO + hq + (size_t)i * d;
+                double m = score_row(&s, Q + hq, K + hk, i, P);
+                double L = softmax_row(&s, P, m);
+                double Di = 0.0;
+                for (int j = 0; j < Nk; ++j)
+                    if (P[j] != 0.0) Di += P[j] * dot(doi, V + hk + (size_t)j * d, d);
+                lse[(size_t)h * Nq + i] = L;
+                Dv[(size_t)h * Nq + i] = Di;
+            }
+        free(P);
+    }
+
+    /* one key column at a time */
+    if (err == OR_OK) {
+#pragma omp parallel for schedule(dynamic, 1)
+        for (int c = 0; c < ncols; ++c) {
+            const int h = head[c], j = col[c];
+            const size_t hq = (size_t)h * Nq * d, hk = (size_t)h * Nk * d;
+            const double *kj = K + hk + (size_t)j * d;
+            const double *vj = V + hk + (size_t)j * d;
+            double *gk = dK + (size_t)c * d;
+            double *gv = dV + (size_t)c * d;
+            for (int k = 0; k < d; ++k) { gk[k] = 0.0; gv[k] = 0.0; }
+            for (int i = 0; i < Nq; ++i) {
+                if (!allowed(&s, i, j)) continue;
+                const double L = lse[(size_t)h * Nq + i];
+                if (L == -INFINITY) continue;
+                const double *qi = Q + hq + (size_t)i * d;
+                const double *doi = dO + hq + (size_t)i * d;
+                const double pij = exp(s.scale * dot(qi, kj, d) - L);
+                const double dpij = dot(doi, vj, d);
+                const double dsij = pij * (dpij - Dv[(size_t)h * Nq + i]);
+                for (int k = 0; k < d; ++k) {
+                    gv[k] += pij * doi[k];
+                    gk[k] += dsij * qi[k];
+                }
+            }
+            for (int k = 0; k < d; ++k) gk[k] *= scale;
+        }
+    }
+    free(need);
+    free(lse);
+    free(Dv);
+    return err;
+}
+
 /* Full probability matrix P [BH,Nq,Nk] (small sizes only). */
 int oracle_probs_qk(const double *Q, const double *K, int BH, int Nq, int Nk, int d, int kind,
                     const uint8_t *block_mask, int block, double scale, double *P)

@@ -107,10 +107,12 @@ def test_bwd_workloads_one_head(name):
 @pytest.mark.parametrize("name", workloads.ORDER)
 def test_bwd_workloads_every_head(name):
     """Full-size workloads in the benchmark's launch configuration, checked
-    in every head: sampled dQ rows (first, last and tile-boundary rows among
-    them) against the oracle's per-row gradient, and dK, dV through the
-    identities sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i (rows of dS sum to
-    zero, rows of P to one; every query row of these workloads sees a key)."""
+    element by element in every head: sampled dQ rows against the oracle's
+    per-row gradient, and sampled dK, dV key rows against its per-key-column
+    gradient (first, last and tile-boundary rows and keys among them); plus
+    the identities sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i over every key
+    (rows of dS sum to zero, rows of P to one; every query row of these
+    workloads sees a key)."""
     w = workloads.WORKLOADS[name]
     x = workloads.make_inputs(w, 3)
     dQ, dK, dV = run(w, x)
@@ -128,6 +130,17 @@ def test_bwd_workloads_every_head(name):
     ref = dQs.reshape(BH, per, w.d)
     for h in range(BH):
         assert_grad(g[h], ref[h], "dQ", f"{name} head {h}")
+    keys = rng.integers(0, w.N, (BH, per))
+    keys[:, 0], keys[:, 1] = 0, w.N - 1
+    keys[:, 2], keys[:, 3] = min(127, w.N - 1), min(128, w.N - 1)
+    keys = keys.reshape(-1)
+    dKs, dVs = oracle.cols(x["Q"], x["K"], x["V"], x["dO"], heads, keys, mask_kind=w.mask,
+                           block_mask=x["mask"], scale=w.scale)
+    for nm, gt, rf in (("dK", dK, dKs), ("dV", dV, dVs)):
+        got = f64(gt).reshape(BH, w.N, w.d)[heads, keys].reshape(BH, per, w.d)
+        rf = rf.reshape(BH, per, w.d)
+        for h in range(BH):
+            assert_grad(got[h], rf[h], nm, f"{name} head {h}")
     dk = f64(dK).reshape(BH, w.N, w.d)
     dv = f64(dV).reshape(BH, w.N, w.d)
     do = f64(x["dO"]).reshape(BH, w.N, w.d)

@@ -49,6 +49,13 @@ MUTANTS = [
     # the single-row path used for sampled parity at full size
     ("rows_dS_sign", "double ds = P[j] * (dot(doi, V + hk + (size_t)j * d, d) - Di);",
      "double ds = P[j] * (dot(doi, V + hk + (size_t)j * d, d) + Di);"),
+    # the key-column path used for sampled dK, dV parity at full size
+    ("cols_dS_sign", "const double dsij = pij * (dpij - Dv[(size_t)h * Nq + i]);",
+     "const double dsij = pij * (dpij + Dv[(size_t)h * Nq + i]);"),
+    ("cols_dV_uses_dS", "gv[k] += pij * doi[k];", "gv[k] += dsij * doi[k];"),
+    ("cols_D_without_P", "if (P[j] != 0.0) Di += P[j] * dot(doi, V + hk + (size_t)j * d, d);\n                lse",
+     "if (P[j] != 0.0) Di += dot(doi, V + hk + (size_t)j * d, d);\n                lse"),
+    ("cols_scale_dropped", "for (int k = 0; k < d; ++k) gk[k] *= scale;", ""),
 ]
 
 # The pins each mutant is run against (all cheap).
@@ -68,6 +75,7 @@ PIN_CALLS = [
     ("cross_more_queries", lambda gd: pins.test_cross_causal_more_queries_than_keys()),
     ("cross_block", lambda gd: pins.test_cross_block_mask_is_query_blocks_by_key_blocks()),
     ("rows_block", lambda gd: pins.test_row_path_matches_full_path("block")),
+    ("cols_block", lambda gd: pins.test_col_path_matches_full_path("block")),
 ]
 
 

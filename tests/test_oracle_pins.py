@@ -272,6 +272,47 @@ def test_row_path_matches_full_path(kind):
         np.testing.assert_allclose(dQ[r], fdQ[h, i], atol=1e-13)
 
 
+@pytest.mark.parametrize("kind", KINDS)
+def test_col_path_matches_full_path(kind):
+    """The key-column sampler (used for sampled dK, dV parity at full size)
+    against the full backward: first, last and tile-boundary keys, repeated
+    heads and keys in any order."""
+    B, H, N, d, block = 2, 2, 260, 32, 128
+    q, k, v, do = (rnd((B, H, N, d), s) for s in (54, 55, 56, 57))
+    bm = small_mask(N, block, 58) if kind == "block" else None
+    g = oracle.bwd(q, k, v, do, kind, bm, 0.2, block=block)
+    heads = [0, 1, 3, 2, 3, 0, 3]
+    keys = [0, 259, 128, 77, 127, 259, 0]
+    dK, dV = oracle.cols(q, k, v, do, heads, keys, mask_kind=kind, block_mask=bm, scale=0.2, block=block)
+    fdK = g["dK"].reshape(B * H, N, d)
+    fdV = g["dV"].reshape(B * H, N, d)
+    for c, (h, j) in enumerate(zip(heads, keys)):
+        np.testing.assert_allclose(dK[c], fdK[h, j], atol=1e-13)
+        np.testing.assert_allclose(dV[c], fdV[h, j], atol=1e-13)
+
+
+@pytest.mark.parametrize("Nq,Nk", [(77, 160), (160, 77)])
+def test_col_path_against_torch_sdpa_fp64(Nq, Nk):
+    """The key-column sampler against PyTorch's fp64 attention + autograd
+    (bottom-right causal through torch.tril, queries and keys of different
+    counts), independently of the oracle's full backward."""
+    d, scale = 16, 0.3
+    g = torch.Generator().manual_seed(80)
+    q, do = (torch.randn((1, 2, Nq, d), generator=g, dtype=torch.float64) for _ in range(2))
+    k, v = (torch.randn((1, 2, Nk, d), generator=g, dtype=torch.float64) for _ in range(2))
+    qt, kt, vt = (t.clone().requires_grad_(True) for t in (q, k, v))
+    am = torch.ones(Nq, Nk, dtype=torch.bool).tril(diagonal=Nk - Nq)
+    live = am.any(dim=1)
+    out = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=am, scale=scale)
+    (out[:, :, live] * do[:, :, live]).sum().backward()
+    heads = [0, 1, 1, 0]
+    keys = [0, Nk - 1, Nk // 2, 63]
+    dK, dV = oracle.cols(q, k, v, do * live[None, None, :, None], heads, keys, mask_kind="causal", scale=scale)
+    for c, (h, j) in enumerate(zip(heads, keys)):
+        np.testing.assert_allclose(dK[c], kt.grad[0, h, j].numpy(), atol=1e-10)
+        np.testing.assert_allclose(dV[c], vt.grad[0, h, j].numpy(), atol=1e-10)
+
+
 def test_bf16_inputs_are_widened_exactly():
     w = workloads.WORKLOADS["tiny"]
     x = workloads.make_inputs(w, seed=0)

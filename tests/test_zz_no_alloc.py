@@ -45,6 +45,11 @@ def test_static_workspace_refuses_problems_that_do_not_fit():
 @pytest.mark.parametrize("shape", [(2, 3, 300, 64, "causal"), (1, 4, 1024, 128, "none"),
                                    (1, 8, 2048, 64, "block")])
 def test_static_workspace_matches_fa_bwd_twice(shape):
+    """Two calls in a row against fa_bwd with a caller-allocated workspace.
+    dK and dV are sums in a fixed order (no atomics), so they must be equal
+    bit for bit; dQ's bulk reduce-adds land in no fixed order, so it is held
+    to the gradient tolerance.  The device's free memory must not move across
+    the second call: the array was reserved by the first one."""
     B, H, N, d, m = shape
     w = workloads.Workload("t", B, H, N, d, m, float(np.float32(d ** -0.5)))
     assert fa.bwd_workspace_size(B, H, N, d) <= MAX_BYTES
@@ -55,8 +60,13 @@ def test_static_workspace_matches_fa_bwd_twice(shape):
     torch.cuda.synchronize()
     for call in range(2):
         got = [torch.full_like(t, float("nan")) for t in want]
+        torch.cuda.synchronize()
+        free_before = torch.cuda.mem_get_info()[0]
         assert call_static(dev, O, L, w, *got) == 0
         assert fa.device_status() == 0
-        for name, g, r in zip(("dQ", "dK", "dV"), got, want):
-            err = rel_l2(f64(g), f64(r))
-            assert err <= GRAD_REL_L2, f"call {call} {name} rel-L2 {err:.3e}"
+        if call == 1:
+            assert torch.cuda.mem_get_info()[0] == free_before, "the second call changed free device memory"
+        err = rel_l2(f64(got[0]), f64(want[0]))
+        assert err <= GRAD_REL_L2, f"call {call} dQ rel-L2 {err:.3e}"
+        for name, g, r in zip(("dK", "dV"), got[1:], want[1:]):
+            assert torch.equal(g, r), f"call {call} {name} differs from fa_bwd"
