@@ -214,6 +214,102 @@ def workload_config(w):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "mask": w.mask, "scale": w.scale}
 
 
+def time_other_workloads(fa, dev, stream, peaks, names, reps=100, seed=0):
+    """Forward and forward + backward of each named workload on the same GPU,
+    in the same run as the headline: the median of `reps` individually timed
+    repetitions (CUDA events on the launching stream).  Workloads whose step
+    touches less than twice the L2 are also timed with the L2 flushed before
+    every repetition (a 2 x L2 buffer written outside the event pair), and
+    that number is the one reported; the warm-L2 figure is kept beside it.
+    Achieved HBM GB/s is the algorithmic bytes (forward: read Q, K, V, write
+    O and LSE; backward: read Q, K, V, O, dO, LSE and D, write dQ, dK, dV)
+    over the time."""
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    out = {}
+    for name in names:
+        w = workloads.WORKLOADS[name]
+        x = workloads.make_inputs(w, seed)
+        Q, K, V, dO = (x[n].to(dev) for n in ("Q", "K", "V", "dO"))
+        mask = x["mask"].to(dev) if x["mask"] is not None else None
+        O = torch.empty_like(Q)
+        LSE = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+        dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+        ws = torch.empty(fa.bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+
+        def fwd():
+            fa.fwd(Q, K, V, w.mask, mask, w.scale, O=O, LSE=LSE, stream=stream)
+
+        def fwd_bwd():
+            fwd()
+            for s in range(3):
+                fa.bwd_stage(s, Q, K, V, O, dO, LSE, dQ, dK, dV, ws, w.mask, mask, w.scale, stream=stream)
+
+        touched = sum(t.numel() * t.element_size() for t in (Q, K, V, dO, O, LSE, dQ, dK, dV)) + ws.numel()
+        modes = ("flushed", "warm") if touched < 2 * L2_BYTES else ("warm",)
+        res = {}
+        for kind, run in (("fwd", fwd), ("fwd_bwd", fwd_bwd)):
+            for _ in range(5):
+                run()
+            torch.cuda.synchronize(dev)
+            for mode in modes:
+                times = []
+                for _ in range(reps):
+                    if mode == "flushed":
+                        flush.fill_(1)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    run()
+                    e1.record(stream)
+                    times.append((e0, e1))
+                torch.cuda.synchronize(dev)
+                res.setdefault(kind, {})[mode] = statistics.median(a.elapsed_time(b) for a, b in times)
+        status = fa.device_status()
+        fl = flops(w, x["mask"])
+        T = w.B * w.H * w.N * w.d
+        rows = w.B * w.H * w.N
+        fwd_bytes = 8 * T + 4 * rows
+        bwd_bytes = 16 * T + 8 * rows
+        rec = {"config": workload_config(w), "l2": "flushed before each repetition" if "flushed" in modes else
+               f"no flush: step touches {touched / 2**20:.0f} MiB, more than twice the L2", "reps": reps,
+               "device_status": status}
+        for kind, fkey, nbytes in (("fwd", ("fwd",), fwd_bytes), ("fwd_bwd", ("fwd", "bwd"), fwd_bytes + bwd_bytes)):
+            ms = res[kind][modes[0]]
+            tf = sum(fl[k] for k in fkey) / (ms * 1e-3) / 1e12
+            rec[kind] = {"ms": ms, "tflops": tf, "frac_of_peak": tf / peaks["bf16_tflops"],
+                         "frac_of_sustained": tf / peaks["bf16_tflops_sustained"],
+                         "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
+                         "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+            if len(modes) == 2:
+                rec[kind]["ms_warm_l2"] = res[kind]["warm"]
+        out[name] = rec
+        del Q, K, V, dO, O, LSE, dQ, dK, dV, ws
+    del flush
+    return out
+
+
+def long_run(step, stream, dev, min_seconds=1.0):
+    """The headline step repeated back to back for at least `min_seconds`
+    (CUDA events around the whole run), with the SM clock sampled: the
+    sustained counterpart of the K-step figure, which a short run takes
+    before the board reaches its power limit."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    n = max(10, int(math.ceil(min_seconds * 1e3 / max(e0.elapsed_time(e1), 1e-3))))
+    clocks = ClockSampler(dev.index)
+    torch.cuda.synchronize(dev)
+    clocks.mark_start()
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark_end()
+    return n, e0.elapsed_time(e1) / n, clocks.result()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -224,6 +320,10 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sustained-run", action="store_true",
+                    help="skip the one-second repeat of the headline step")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the per-workload timing of the other configurations")
     ap.add_argument("--vs-standard", action="store_true",
                     help="time the fused forward against standard (materialising) attention instead")
     args = ap.parse_args()
@@ -389,6 +489,21 @@ def main():
                                    fl["fwd"] + fl["bwd"])
     status = status or fa.device_status()
 
+    # ---- the same step repeated for at least a second (sustained clocks)
+    sustained = None
+    if not args.no_sustained_run:
+        n_long, ms_long, clocks_long = long_run(step, stream, dev)
+        sustained = {"steps": n_long, "ms_per_step": ms_long,
+                     "tflops": (fl["fwd"] + fl["bwd"]) / (ms_long * 1e-3) / 1e12, "clocks": clocks_long}
+        sustained["frac_of_peak"] = sustained["tflops"] / peaks["bf16_tflops"]
+        sustained["frac_of_sustained"] = sustained["tflops"] / peaks["bf16_tflops_sustained"]
+
+    # ---- the other configurations, on the same GPU (single-GPU runs only)
+    others = None
+    if world == 1 and not args.no_other_workloads:
+        others = time_other_workloads(fa, dev, stream, peaks, [n for n in workloads.ORDER if n != w.name])
+        status = status or max(r["device_status"] for r in others.values())
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, dt, desc, cores = cpu_baseline(w, x, mask_cpu)
@@ -403,8 +518,10 @@ def main():
         "config": dict(workload_config(w), parallelism=f"{world} independent replica(s), one per GPU",
                        l2=f"no flush: step touches {in_bytes / 2**20:.0f} MiB, more than the "
                           f"{L2_BYTES / 2**20:.0f} MiB L2"),
-        "fwd": {"ms": per_kernel["fwd"], "tflops": fwd_tflops, "frac_of_peak": fwd_tflops / peaks["bf16_tflops"]},
-        "fwd_bwd": {"ms": ms_step, "tflops": value / world, "frac_of_peak": value / world / peaks["bf16_tflops"]},
+        "fwd": {"ms": per_kernel["fwd"], "tflops": fwd_tflops, "frac_of_peak": fwd_tflops / peaks["bf16_tflops"],
+                "frac_of_sustained": fwd_tflops / peaks["bf16_tflops_sustained"]},
+        "fwd_bwd": {"ms": ms_step, "tflops": value / world, "frac_of_peak": value / world / peaks["bf16_tflops"],
+                    "frac_of_sustained": value / world / peaks["bf16_tflops_sustained"]},
         "bwd": {"ms": bwd_ms, "tflops": bwd_tflops},
         "kernels_ms": per_kernel,
         "roofline": roofline,
@@ -415,6 +532,8 @@ def main():
                             "streams during step i's compute"},
         "gpu_launches": 4 * args.steps,
         "clocks": clock_info,
+        "sustained_run": sustained,
+        "per_workload": others,
         "device_status": status,
         "peaks": {"bf16_tflops": peaks["bf16_tflops"], "bf16_tflops_sustained": peaks["bf16_tflops_sustained"],
                   "source": peak_kind},
