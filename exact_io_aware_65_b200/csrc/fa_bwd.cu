@@ -441,18 +441,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t IDESC_T = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T: K-major A and B
       constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, 0, 1);    // dV, dK: A in TMEM, B MN-major
       constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, 1, 1);    // dQ: both MN-major
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aDS = smem_u32(sDS), aQD = smem_u32(sQD);
       uint32_t item_iter = 0, qd_iter = 0, dq_iter = 0, p_cnt = 0, ds_cnt = 0;
       bool ok = true, issued = false;
+      // Descriptors built once; the products below only move them (one
+      // 32-bit add per operand).  K-major forms (K = d) for the score
+      // products, MN-major forms for the gradient products.
+      const Desc kK = desc_sw128(smem_u32(sK), 16, 1024), kV = desc_sw128(smem_u32(sV), 16, 1024);
+      const Desc kQD = desc_sw128(smem_u32(sQD), 16, 1024);
+      const Desc mQD = desc_sw128(smem_u32(sQD), C::CHUNK_BYTES, 1024);
+      const Desc mDS = desc_sw128(smem_u32(sDS), C::CHUNK_BYTES, 1024);
+      const Desc mK = desc_sw128(smem_u32(sK), C::CHUNK_BYTES, 1024);
 
       // S^T = K Q^T into the score columns (M = keys, N = queries, K = d).
       auto issue_s = [&](uint32_t st) {
-        const uint32_t aQ = aQD + st * 2 * C::TILE_BYTES;
+        const Desc q = desc_at(kQD, st * 2 * C::TILE_BYTES);
 #pragma unroll
         for (int s = 0; s < D / 16; ++s) {
           const uint32_t off = (s >> 2) * C::CHUNK_BYTES + (s & 3) * 32;
-          mma_ss(tmem + C::COL_S, smem_desc_sw128(aK + off, 16, 1024), smem_desc_sw128(aQ + off, 16, 1024),
-                 IDESC_T, s > 0 ? 1u : 0u);
+          mma_ss(tmem + C::COL_S, desc_at(kK, off), desc_at(q, off), IDESC_T, s > 0 ? 1u : 0u);
         }
         tc_commit(&s_full);
       };
@@ -465,12 +471,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!mbar_wait(&dq_free[0], (dq_iter - 1) & 1, w)) return false;
         }
         tc_fence_after();
-        const uint32_t adO = aQD + st * 2 * C::TILE_BYTES + C::TILE_BYTES;
+        const Desc dO = desc_at(kQD, st * 2 * C::TILE_BYTES + C::TILE_BYTES);
 #pragma unroll
         for (int s = 0; s < D / 16; ++s) {
           const uint32_t off = (s >> 2) * C::CHUNK_BYTES + (s & 3) * 32;
-          mma_ss(tmem + C::COL_DP, smem_desc_sw128(aV + off, 16, 1024), smem_desc_sw128(adO + off, 16, 1024),
-                 IDESC_T, s > 0 ? 1u : 0u);
+          mma_ss(tmem + C::COL_DP, desc_at(kV, off), desc_at(dO, off), IDESC_T, s > 0 ? 1u : 0u);
         }
         tc_commit(&dp_full);
         return true;
@@ -497,8 +502,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int inext = next_q<VARLEN>(p, it, i + 1);
           const uint32_t st = qd_iter % C::NST;         // stage of query tile i
           const uint32_t stn = (qd_iter + 1) % C::NST;  // stage of query tile inext
-          const uint32_t aQ = aQD + st * 2 * C::TILE_BYTES;
-          const uint32_t adO = aQ + C::TILE_BYTES;
+          const Desc gQ = desc_at(mQD, st * 2 * C::TILE_BYTES);  // MN-major Q of tile i
+          const Desc gdO = desc_at(gQ, C::TILE_BYTES);          // MN-major dO of tile i
           // dV += P^T dO (A = P^T in TMEM, K = 128 queries)
           ok = mbar_wait(&p_full, p_cnt & 1, w);
           if (!ok) break;
@@ -506,8 +511,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
 #pragma unroll
           for (int s = 0; s < BQ / 16; ++s)
-            mma_ts(tmem + C::COL_DV, tmem + C::COL_P + s * 8, smem_desc_sw128(adO + s * 2048, C::CHUNK_BYTES, 1024),
-                   IDESC_G, (n > 0 || s > 0) ? 1u : 0u);
+            mma_ts(tmem + C::COL_DV, tmem + C::COL_P + s * 8, desc_at(gdO, s * 2048), IDESC_G,
+                   (n > 0 || s > 0) ? 1u : 0u);
           // S^T of the next query tile goes in now: its columns were last read
           // by the dV product just issued, and its softmax can then overlap
           // the dK, dQ and next dP products.
@@ -524,8 +529,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
 #pragma unroll
           for (int s = 0; s < BQ / 16; ++s)
-            mma_ts(tmem + C::COL_DK, tmem + C::COL_DS + s * 8, smem_desc_sw128(aQ + s * 2048, C::CHUNK_BYTES, 1024),
-                   IDESC_G, (n > 0 || s > 0) ? 1u : 0u);
+            mma_ts(tmem + C::COL_DK, tmem + C::COL_DS + s * 8, desc_at(gQ, s * 2048), IDESC_G,
+                   (n > 0 || s > 0) ? 1u : 0u);
           const uint32_t b = dq_iter % C::NDQ;
           if (D == 64 && dq_iter >= (uint32_t)C::NDQ) {
             ok = mbar_wait(&dq_free[b], ((dq_iter / C::NDQ) - 1) & 1, w);
@@ -534,8 +539,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
 #pragma unroll
           for (int s = 0; s < BK / 16; ++s)
-            mma_ss(tmem + C::col_dq(b), smem_desc_sw128(aDS + s * 2048, C::CHUNK_BYTES, 1024),
-                   smem_desc_sw128(aK + s * 2048, C::CHUNK_BYTES, 1024), IDESC_Q, s > 0 ? 1u : 0u);
+            mma_ss(tmem + C::col_dq(b), desc_at(mDS, s * 2048), desc_at(mK, s * 2048), IDESC_Q, s > 0 ? 1u : 0u);
           tc_commit(&dq_full[b]);
           if (C::DQ_PARTS == 2) tc_commit(&q_empty[st]);  // the rest goes back via the dQ drain
           ++qd_iter;

@@ -232,25 +232,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t kv_iter = 0, item_iter = 0, p_cnt[2] = {0, 0};
       bool ok = true, issued = false;
 
+      // Descriptors of the Q tiles and of ring slot 0, built once; the
+      // products below only move them (one 32-bit add per operand).
+      const Desc dQ0 = desc_sw128(sQ_addr, 16, 1024);             // K-major, K = d
+      const Desc dK0 = desc_sw128(sKV_addr, 16, 1024);            // K-major, K = d
+      const Desc dV0 = desc_sw128(sKV_addr, C::CHUNK_BYTES, 1024);  // MN-major, N = d
       auto issue_s = [&](int t, uint32_t kslot) {
-        const uint32_t qa = sQ_addr + t * C::TILE_BYTES;
-        const uint32_t ka = sKV_addr + kslot * C::TILE_BYTES;
+        const Desc qa = desc_at(dQ0, t * C::TILE_BYTES);
+        const Desc ka = desc_at(dK0, kslot * C::TILE_BYTES);
+        const uint32_t d_s = tmem + t * 128;
 #pragma unroll
         for (int s = 0; s < D / 16; ++s) {
           const uint32_t off = (s >> 2) * C::CHUNK_BYTES + (s & 3) * 32;
-          mma_ss(tmem + t * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), IDESC_S,
-                 s > 0 ? 1u : 0u);
+          mma_ss(d_s, desc_at(qa, off), desc_at(ka, off), IDESC_S, s > 0 ? 1u : 0u);
         }
         tc_commit(&s_full[t]);
         issued = true;
       };
       auto issue_pv = [&](int t, uint32_t vslot, uint32_t acc) {
-        const uint32_t va = sKV_addr + vslot * C::TILE_BYTES;
+        const Desc va = desc_at(dV0, vslot * C::TILE_BYTES);
+        const uint32_t d_o = tmem + 256 + t * D, a_p = tmem + t * 128;
 #pragma unroll
-        for (int s = 0; s < BN / 16; ++s) {
-          mma_ts(tmem + 256 + t * D, tmem + t * 128 + s * 8, smem_desc_sw128(va + s * 2048, C::CHUNK_BYTES, 1024),
-                 IDESC_O, (s > 0 || acc) ? 1u : 0u);
-        }
+        for (int s = 0; s < BN / 16; ++s)
+          mma_ts(d_o, a_p + s * 8, desc_at(va, s * 2048), IDESC_O, (s > 0 || acc) ? 1u : 0u);
       };
 
       for (;; ++item_iter) {

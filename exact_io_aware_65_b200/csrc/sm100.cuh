@@ -268,6 +268,42 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t smem_addr, uint32_t
   return d;
 }
 
+// The issuers keep a descriptor as its two 32-bit words.  The start address
+// occupies the low 14 bits of the low word, in 16-byte units, and a shared
+// memory address stays below 256 KB, so moving a descriptor by a byte offset
+// inside its buffer is one 32-bit add of (offset >> 4) to the low word, with
+// no carry into the other fields.  The MMA issuer shares its SM sub-partition
+// with busy softmax warps, so the fewer instructions it spends per MMA the
+// sooner the tensor cores see the next one.
+struct Desc {
+  uint32_t lo, hi;
+};
+__device__ __forceinline__ Desc desc_sw128(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  const uint64_t d = smem_desc_sw128(smem_addr, lbo_bytes, sbo_bytes);
+  return Desc{uint32_t(d), uint32_t(d >> 32)};
+}
+__device__ __forceinline__ Desc desc_at(Desc d, uint32_t byte_off) { return Desc{d.lo + (byte_off >> 4), d.hi}; }
+
+// mma_ss / mma_ts with the descriptors as word pairs.
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, Desc a, Desc b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}"
+      ::"r"(d_tmem), "r"(a.lo), "r"(a.hi), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, Desc b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "r"(b.lo), "r"(b.hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // TMEM loads/stores: 32 lanes x 32 bits, repeated over consecutive columns.
 // Thread i of the warp reads/writes lane (warp's lane quarter base + i).
 #define FA_TMEM_LD_X32(taddr, r)                                                                        \
