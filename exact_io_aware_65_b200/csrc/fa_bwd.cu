@@ -282,6 +282,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // part h; dq_half: the first part has been read out).  One barrier per
   // part, each completing one phase per tile.
   __shared__ __align__(8) uint64_t dq_staged[2], dq_half;
+  // d = 128, unordered dQ: the second half of a dQ tile is staged in the dS
+  // buffer (free once the tile's dQ product has read it), so both halves
+  // are in flight at once.  dss_full: the softmax has written dS to shared
+  // memory (the dQ product may read it); sds_free: the drain's bulk read of
+  // the half staged there is done (the softmax may write the next dS).
+  __shared__ __align__(8) uint64_t dss_full, sds_free;
   // Each stage holds a query tile's Q (with its LSE values) and dO (with its
   // D values), filled and released independently: the dQ drain releases
   // what held the tile's dQ for its bulk reduction, the MMA warp the Q half
@@ -311,6 +317,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(&dq_staged[0], 128);
     mbar_init(&dq_staged[1], 128);
     mbar_init(&dq_half, 1);
+    mbar_init(&dss_full, 256);
+    mbar_init(&sds_free, 1);
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
@@ -441,7 +449,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t IDESC_T = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T: K-major A and B
       constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, 0, 1);    // dV, dK: A in TMEM, B MN-major
       constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, 1, 1);    // dQ: both MN-major
-      uint32_t item_iter = 0, qd_iter = 0, dq_iter = 0, p_cnt = 0, ds_cnt = 0;
+      uint32_t item_iter = 0, qd_iter = 0, dq_iter = 0, p_cnt = 0, ds_cnt = 0, dss_cnt = 0;
       bool ok = true, issued = false;
       // Descriptors built once; the products below only move them (one
       // 32-bit add per operand).  K-major forms (K = d) for the score
@@ -537,6 +545,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!ok) break;
             tc_fence_after();
           }
+          ok = mbar_wait(&dss_full, dss_cnt & 1, w);  // dS in shared memory
+          if (!ok) break;
+          ++dss_cnt;
 #pragma unroll
           for (int s = 0; s < BK / 16; ++s)
             mma_ss(tmem + C::col_dq(b), desc_at(mDS, s * 2048), desc_at(mK, s * 2048), IDESC_Q, s > 0 ? 1u : 0u);
@@ -654,14 +665,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             dk[cc * 16 + u * 2 + 1] = pack_bf16x2(g2, g3);
           }
         }
-        // Shared-memory copy of dS^T (the A operand of dQ = dS K), 128-byte
-        // swizzle: 16-byte unit u of row kr lives at unit (u ^ (kr & 7)).
-        uint8_t* ds_row = sDS + hf * C::CHUNK_BYTES + kr * 128;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int unit = u ^ (kr & 7);
-          *reinterpret_cast<uint4*>(ds_row + unit * 16) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
-        }
         // dS^T overwrites dP^T columns the other column half may still be
         // reading: wait until both halves have loaded theirs.
         ok = mbar_wait_warp(&dp_read, par, w);
@@ -669,9 +672,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         FA_TMEM_ST_X32(tmem + lane_bits + C::COL_DS + hf * 32, dk);
         tc_wait_st();
-        fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&ds_full);
+        mbar_arrive(&ds_full);  // dK may start
+        // Shared-memory copy of dS^T (the A operand of dQ = dS K), 128-byte
+        // swizzle: 16-byte unit u of row kr lives at unit (u ^ (kr & 7)).
+        // With the split drain the buffer may still hold half of the
+        // previous dQ tile on its way to the accumulator.
+        if (D == 128 && !p.deterministic && s_cnt > 1) {
+          ok = mbar_wait_warp(&sds_free, (s_cnt - 2) & 1, w);
+          if (!ok) break;
+        }
+        uint8_t* ds_row = sDS + hf * C::CHUNK_BYTES + kr * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int unit = u ^ (kr & 7);
+          *reinterpret_cast<uint4*>(ds_row + unit * 16) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&dss_full);
         any = true;
       }
       if (!ok) break;
@@ -729,9 +747,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ok = mbar_wait_warp(&dq_full[b], (dq_iter / C::NDQ) & 1, w);
         if (!ok) break;
         tc_fence_after();
+        // With the split drain (d = 128, unordered) columns 64..127 are
+        // staged first: they go to v[0, 64) and columns 0..63 to v[64, 128).
+        const bool split = D == 128 && !p.deterministic;
         uint32_t v[D];
 #pragma unroll
-        for (int c = 0; c < D; c += 32) FA_TMEM_LD_X32(tmem + lane_bits + C::col_dq(b) + c, (v + c));
+        for (int c = 0; c < D; c += 32)
+          FA_TMEM_LD_X32(tmem + lane_bits + C::col_dq(b) + (split ? (c + D / 2) % D : c), (v + c));
         tc_wait_ld();
         tc_fence_before();
         mbar_arrive(&dq_free[b]);
@@ -742,6 +764,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         constexpr int GROUPS = D / 4 / C::DQ_PARTS;  // 4-column groups per part
         uint8_t* slot = sQD + st * 2 * C::TILE_BYTES + C::DQ_SLOT_OFF;
         float* dst = p.dq_acc + ((size_t)it.bh * p.Npad + (size_t)i * BQ) * D;
+        if (D == 128 && !p.deterministic) {
+          // Both halves in flight at once: columns 64..127 staged in the dS
+          // buffer (its dQ product has completed) and added first, columns
+          // 0..63 in the tile's dO half.  The dS buffer goes back to the
+          // softmax once its half has been read, the dO half to the producer
+          // once the second has.
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            // h = 0: columns 64..127 (v[0, 64)) into the dS buffer;
+            // h = 1: columns 0..63 (v[64, 128)) into the dO half
+            uint8_t* buf = h == 0 ? sDS : slot;
+            const int part = 1 - h;  // which half of the accumulator tile
+#pragma unroll
+            for (int e = 0; e < GROUPS; ++e) {
+              const int g = h * GROUPS + e;
+              *reinterpret_cast<uint4*>(buf + e * 2048 + qr * 16) =
+                  make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+            }
+            fence_proxy_async_smem();
+            // a warp that has run ahead arrives only once the previous
+            // tile's phase of this barrier is complete
+            if (dq_iter > 0) {
+              ok = mbar_wait_warp(&dq_staged[h], (dq_iter - 1) & 1, w);
+              if (!ok) break;
+            }
+            mbar_arrive(&dq_staged[h]);
+            if (leader) {
+              ok = mbar_wait(&dq_staged[h], dq_iter & 1, w);
+              if (ok && FA_IN_BOUNDS(p.status, ((size_t)it.bh * p.Npad + (size_t)i * BQ) * D + part * GROUPS * 512,
+                                     C::DQ_PART_BYTES / 4, (size_t)p.BH * p.Npad * D))
+                bulk_reduce_add_f32(dst + part * GROUPS * 512, buf, C::DQ_PART_BYTES);
+              bulk_commit_group();
+              bulk_issued = true;
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+          }
+          if (!ok) break;
+          if (leader) {
+            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");  // the dS-buffer half
+            mbar_arrive(&sds_free);
+            bulk_wait_read_all();
+            mbar_arrive(&do_empty[st]);
+          }
+          __syncwarp();
+          ++dq_iter;
+          continue;
+        }
 #pragma unroll
         for (int h = 0; h < C::DQ_PARTS; ++h) {
           if (h == 1) {
