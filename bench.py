@@ -210,6 +210,28 @@ def throughput(total_ms: float, steps: int, world: int, flops_per_step: float) -
     return ms, world * flops_per_step / (ms * 1e-3) / 1e12
 
 
+def head_range(heads: int, world: int, rank: int) -> tuple:
+    """Contiguous range [h0, h1) of the flattened B*H heads that `rank` takes
+    when one problem is split across `world` ranks by heads.  Heads are
+    independent in both passes, so the split needs no collective; ranges
+    differ in length by at most one head."""
+    if heads < world:
+        raise ValueError(f"{heads} heads cannot be split over {world} ranks")
+    return rank * heads // world, (rank + 1) * heads // world
+
+
+def slice_heads(x: dict, w, h0: int, h1: int) -> dict:
+    """The rank's part of the problem: heads [h0, h1) of Q, K, V and dO as
+    contiguous [1, h1 - h0, N, d] tensors; the block mask is shared by every
+    head and is kept whole."""
+    out = {}
+    for n in ("Q", "K", "V", "dO"):
+        t = x[n].reshape(w.B * w.H, w.N, w.d)[h0:h1]
+        out[n] = t.reshape(1, h1 - h0, w.N, w.d).contiguous()
+    out["mask"] = x["mask"]
+    return out
+
+
 def workload_config(w):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "mask": w.mask, "scale": w.scale}
 
@@ -324,6 +346,9 @@ def main():
                     help="skip the one-second repeat of the headline step")
     ap.add_argument("--no-other-workloads", action="store_true",
                     help="skip the per-workload timing of the other configurations")
+    ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
+                    help="with N > 1: one replica of the workload per rank (weak scaling, default), or one "
+                         "problem split by heads across the ranks (strong scaling, no collective)")
     ap.add_argument("--vs-standard", action="store_true",
                     help="time the fused forward against standard (materialising) attention instead")
     args = ap.parse_args()
@@ -355,8 +380,16 @@ def main():
         if dist is not None:
             dist.barrier()
 
-    # ---- inputs resident in HBM (each rank its own replica of the workload)
-    x = workloads.make_inputs(w, args.seed + rank)
+    # ---- inputs resident in HBM: each rank its own replica of the workload,
+    # or (--split heads) its range of the heads of one problem
+    split = args.split == "heads" and world > 1
+    w_full = w
+    if split:
+        h0, h1 = head_range(w.B * w.H, world, rank)
+        x = slice_heads(workloads.make_inputs(w, args.seed), w, h0, h1)
+        w = w.with_(B=1, H=h1 - h0)
+    else:
+        x = workloads.make_inputs(w, args.seed + rank)
     mask_cpu = x["mask"]
     Q, K, V, dO = (x[n].to(dev) for n in ("Q", "K", "V", "dO"))
     mask = mask_cpu.to(dev) if mask_cpu is not None else None
@@ -402,8 +435,12 @@ def main():
     per_kernel = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(names)}
     clock_info = clocks.result()
 
-    fl = flops(w, mask_cpu)
-    ms_step, value = throughput(total_ms, args.steps, world, fl["fwd"] + fl["bwd"])
+    fl = flops(w, mask_cpu)  # this rank's part
+    fl_job = flops(w_full, mask_cpu)
+    if split:  # one problem: the whole job is the full problem's work in the slowest rank's time
+        ms_step, value = throughput(total_ms, args.steps, 1, fl_job["fwd"] + fl_job["bwd"])
+    else:
+        ms_step, value = throughput(total_ms, args.steps, world, fl["fwd"] + fl["bwd"])
     peaks, peak_kind = load_peaks()
     fwd_tflops = fl["fwd"] / (per_kernel["fwd"] * 1e-3) / 1e12
     bwd_ms = per_kernel["bwd_prep"] + per_kernel["bwd_main"] + per_kernel["bwd_dq_convert"]
@@ -485,13 +522,14 @@ def main():
     e1.record(down)                               # the last download ends after all other work
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms, e2e_value = throughput(max_over_ranks(e0.elapsed_time(e1), dist, dev), e2e_steps, world,
-                                   fl["fwd"] + fl["bwd"])
+    e2e_ms, e2e_value = throughput(max_over_ranks(e0.elapsed_time(e1), dist, dev), e2e_steps,
+                                   1 if split else world,
+                                   (fl_job if split else fl)["fwd"] + (fl_job if split else fl)["bwd"])
     status = status or fa.device_status()
 
     # ---- the same step repeated for at least a second (sustained clocks)
     sustained = None
-    if not args.no_sustained_run:
+    if not args.no_sustained_run and world == 1:
         n_long, ms_long, clocks_long = long_run(step, stream, dev)
         sustained = {"steps": n_long, "ms_per_step": ms_long,
                      "tflops": (fl["fwd"] + fl["bwd"]) / (ms_long * 1e-3) / 1e12, "clocks": clocks_long}
@@ -512,16 +550,20 @@ def main():
     in_bytes = sum(t.numel() * t.element_size() for t in (Q, K, V, dO, O, LSE, dQ, dK, dV)) + ws.numel()
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong" if split else "weak",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded i.i.d. N(0,1) Q, K, V, dO rounded to bf16 (no dataset)",
-        "config": dict(workload_config(w), parallelism=f"{world} independent replica(s), one per GPU",
+        "config": dict(workload_config(w_full),
+                       parallelism=(f"one problem split by heads over {world} GPUs (contiguous head ranges, "
+                                    f"no collective)") if split else f"{world} independent replica(s), one per GPU",
                        l2=f"no flush: step touches {in_bytes / 2**20:.0f} MiB, more than the "
                           f"{L2_BYTES / 2**20:.0f} MiB L2"),
         "fwd": {"ms": per_kernel["fwd"], "tflops": fwd_tflops, "frac_of_peak": fwd_tflops / peaks["bf16_tflops"],
                 "frac_of_sustained": fwd_tflops / peaks["bf16_tflops_sustained"]},
         "fwd_bwd": {"ms": ms_step, "tflops": value / world, "frac_of_peak": value / world / peaks["bf16_tflops"],
-                    "frac_of_sustained": value / world / peaks["bf16_tflops_sustained"]},
+                    "frac_of_sustained": value / world / peaks["bf16_tflops_sustained"],
+                    "per": "GPU (whole-job value / N)"},
         "bwd": {"ms": bwd_ms, "tflops": bwd_tflops},
         "kernels_ms": per_kernel,
         "roofline": roofline,
