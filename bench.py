@@ -236,10 +236,21 @@ def workload_config(w):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "mask": w.mask, "scale": w.scale}
 
 
+def trimmed_mean(xs, cut=0.1):
+    """Mean of xs without the lowest and highest `cut` fraction."""
+    xs = sorted(xs)
+    k = int(len(xs) * cut)
+    kept = xs[k:len(xs) - k] if len(xs) > 2 * k else xs
+    return sum(kept) / len(kept)
+
+
 def time_other_workloads(fa, dev, stream, peaks, names, reps=100, seed=0):
     """Forward and forward + backward of each named workload on the same GPU,
-    in the same run as the headline: the median of `reps` individually timed
-    repetitions (CUDA events on the launching stream).  Workloads whose step
+    in the same run as the headline: the mean of `reps` individually timed
+    repetitions (CUDA events on the launching stream) after dropping the
+    fastest and slowest tenth.  (Event times of short launches come in steps
+    of about 2 us on this part: a median sits on one step, the trimmed mean
+    averages across them.)  Workloads whose step
     touches less than twice the L2 are also timed with the L2 flushed before
     every repetition (a 2 x L2 buffer written outside the event pair), and
     that number is the one reported; the warm-L2 figure is kept beside it.
@@ -284,7 +295,7 @@ def time_other_workloads(fa, dev, stream, peaks, names, reps=100, seed=0):
                     e1.record(stream)
                     times.append((e0, e1))
                 torch.cuda.synchronize(dev)
-                res.setdefault(kind, {})[mode] = statistics.median(a.elapsed_time(b) for a, b in times)
+                res.setdefault(kind, {})[mode] = trimmed_mean([a.elapsed_time(b) for a, b in times])
         status = fa.device_status()
         fl = flops(w, x["mask"])
         T = w.B * w.H * w.N * w.d

@@ -18,16 +18,25 @@
 //                 tensor memory, keeps the row max m and row sum l in
 //                 registers, writes P (bf16) back over the scores, and does
 //                 the final O / l and LSE epilogue.
-// Tensor memory (512 columns): S/P of tile t at [128 t, 128 t + 128), O of
-// tile t at [256 + d t, 256 + d t + d).
+// Tensor memory (512 columns):
+//   d = 128: S/P of tile t at [128 t, 128 t + 128) (P, bf16, over the scores),
+//            O of tile t at [256 + 128 t, 384 + 128 t).  A tile's next QK^T
+//            waits for its PV, which reads P from the same columns; the two
+//            query tiles ping-pong, so while one softmax group works on its
+//            scores the tensor cores run the other tile's PV and next QK^T.
+//   d = 64:  S of tile t at [128 t, 128 t + 128), P of tile t at
+//            [256 + 64 t, 320 + 64 t), O of tile t at [384 + 64 t, 448 + 64 t).
+//            P has columns of its own, so the next QK^T overwrites S as soon
+//            as the softmax has read it (barrier s_free) and the scores of key
+//            tile j + 1 are ready when the softmax finishes tile j: each
+//            softmax group runs its key steps back to back.
 //
-// The two query tiles ping-pong: while one softmax group works on its scores
-// the tensor cores run the other tile's PV and next QK^T products.
-//
-// The O rescale is lazy: the reference maximum used for exponentials only
-// moves when the true maximum has grown by more than 2^8; l and O always use
-// the same reference, so the final O / l is unchanged (exact in exact
-// arithmetic) while most tiles skip the tensor-memory round trip.
+// The O rescale is lazy: each row takes its reference maximum from its first
+// key tile and keeps it while the exponentials stay below 2^16 (a row sum of
+// one key tile below 2^16), so no later key tile needs a row maximum.  A key
+// tile that breaks the bound is redone on its own row maximum and l and O
+// move to the new reference; l and O always share the reference, so the
+// final O / l is unchanged (exact in exact arithmetic).
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -52,7 +61,6 @@ constexpr int RING = 4;              // depth of the item ring the producer fill
 constexpr uint32_t SCHED_SLOTS = 4096;
 __device__ uint32_t g_claim[SCHED_SLOTS];  // dynamic claims so far
 __device__ uint32_t g_done[SCHED_SLOTS];   // CTAs that stopped claiming
-constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 constexpr float LN2 = 0.69314718055994530942f;
 
 template <int D>
@@ -61,7 +69,10 @@ struct Cfg {
   static constexpr int CHUNKS = D / 64;          // 64-column (128-byte) chunks per row
   static constexpr int CHUNK_BYTES = BN * 128;   // one chunk of a tile
   static constexpr int NSLOT = D == 64 ? 8 : 4;  // K/V ring slots
-  static constexpr int SMEM_BYTES = 2 * TILE_BYTES + NSLOT * TILE_BYTES + 1024;
+  // d = 64: each softmax warp stages its 32 rows of O (bf16) here so that
+  // they go out to global memory four whole rows per store instruction.
+  static constexpr int OSTAGE_BYTES = D == 64 ? 8 * 32 * D * 2 : 0;
+  static constexpr int SMEM_BYTES = 2 * TILE_BYTES + NSLOT * TILE_BYTES + OSTAGE_BYTES + 1024;
   // MMA issuer threads.  Issuing blocks while the tensor core's queue is
   // full, so with one issuer a tile's PV can wait behind the other tile's
   // products.  d = 64: one issuer per query tile (short products, so the
@@ -69,7 +80,17 @@ struct Cfg {
   // tile's PV and next QK^T back to back on the tensor core (interleaving
   // the two tiles' products delays both tiles' next scores).
   static constexpr int ISSUERS = D == 64 ? 2 : 1;
+  // P in columns of its own (needs 2 x (128 + 64 + d) <= 512 columns).
+  static constexpr bool SPLIT_P = D == 64;
+  static constexpr uint32_t COL_P = 256;                   // + 64 t (SPLIT_P)
+  static constexpr uint32_t COL_O = SPLIT_P ? 384 : 256;   // + d t
   static constexpr int CONSUMERS = ISSUERS + 8;  // of the item ring: issuers + softmax warps
+  // Registers per thread after the split (launch: 168): producer and issuer
+  // warpgroup, then each softmax warpgroup.  The d = 64 softmax holds a
+  // whole score row and spills below 224.
+  static constexpr int REG_CTL = D == 64 ? 56 : 88;
+  static constexpr int REG_SMX = D == 64 ? 224 : 208;
+  static_assert(REG_CTL + 2 * REG_SMX <= 3 * 168, "register split exceeds the launch");
 };
 
 // VARLEN: per-sequence lengths are read (else every sequence has N, Nk and
@@ -83,10 +104,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                        // 2 tiles
   uint8_t* sKV = smem + 2 * C::TILE_BYTES;   // NSLOT tiles
+  uint8_t* sO = sKV + C::NSLOT * C::TILE_BYTES;  // OSTAGE_BYTES
 
   __shared__ __align__(8) uint64_t q_full, q_empty, mma_drain[2];
   __shared__ __align__(8) uint64_t kv_full[C::NSLOT], kv_empty[C::NSLOT];
   __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_full[2];
+  __shared__ __align__(8) uint64_t s_free[2], pv_done[2];  // SPLIT_P only
   // The producer claims work items and passes them to the other roles.
   __shared__ __align__(8) uint64_t item_full[RING], item_empty[RING];
   __shared__ int item_ring[RING];
@@ -109,6 +132,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], BM);
       mbar_init(&o_full[t], 1);
+      mbar_init(&s_free[t], BM);
+      mbar_init(&pv_done[t], 1);
     }
     for (int r = 0; r < RING; ++r) {
       mbar_init(&item_full[r], 1);
@@ -149,11 +174,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   };
 
   // Registers: 384 threads x 168 at launch; the producer/MMA warpgroup gives
-  // much of its share to the two softmax warpgroups: 128 x (88 + 208 + 208)
-  // = 64512, the launch total.
-  static_assert(88 + 208 + 208 <= 3 * 168, "register split exceeds the launch");
+  // much of its share to the two softmax warpgroups (Cfg::REG_CTL,
+  // Cfg::REG_SMX; 128 x (56 + 224 + 224) = 128 x (88 + 208 + 208) = 64512,
+  // the launch total).
   if (warp < 4) {
-    regs_dec<88>();  // may only lower the 168 registers of the launch
+    regs_dec<C::REG_CTL>();  // may only lower the 168 registers of the launch
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -251,12 +276,77 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       auto issue_pv = [&](int t, uint32_t vslot, uint32_t acc) {
         const Desc va = desc_at(dV0, vslot * C::TILE_BYTES);
-        const uint32_t d_o = tmem + 256 + t * D, a_p = tmem + t * 128;
+        const uint32_t d_o = tmem + C::COL_O + t * D;
+        const uint32_t a_p = tmem + (C::SPLIT_P ? C::COL_P + t * 64 : t * 128);
 #pragma unroll
         for (int s = 0; s < BN / 16; ++s)
           mma_ts(d_o, a_p + s * 8, desc_at(va, s * 2048), IDESC_O, (s > 0 || acc) ? 1u : 0u);
       };
 
+      if constexpr (C::SPLIT_P) {
+        // One tile per issuer.  Per union key step j (K of j at ring index
+        // kv_iter, its V at kv_iter + 1): S = Q K_j^T once the softmax has
+        // read the previous scores, then O += P V for the key tile before j
+        // once its P is written.  Every S, P and PV is counted over the whole
+        // launch, so the n-th of each pairs with the n-th arrival.
+        const int t = warp - 1;
+        uint32_t s_iss = 0, pv_iss = 0;
+        for (;; ++item_iter) {
+          int idx;
+          ok = take_item(item_iter, idx);
+          if (!ok || idx >= p.n_items) break;
+          const Item it = item_at<VARLEN>(p, idx);
+          const bool mine = t == 0 || it.has1;
+          const int qt = t == 0 ? it.q0 : it.q1;
+          ok = mbar_wait(&q_full, item_iter & 1, w);
+          if (!ok) break;
+          tc_fence_after();
+          const int e = kv_end<VARLEN>(p, it);
+          int j = next_union<VARLEN>(p, it, 0), jp = -1;
+          if (j >= e) tc_commit(&q_empty);  // no key tile: Q was not read
+          bool first_pv = true;
+          while (ok && (j < e || jp >= 0)) {
+            const int jn = j < e ? next_union<VARLEN>(p, it, j + 1) : e;
+            if (j < e) {
+              const uint32_t ks = kv_iter % C::NSLOT;
+              ok = mbar_wait(&kv_full[ks], (kv_iter / C::NSLOT) & 1, w);
+              if (!ok) break;
+              tc_fence_after();
+              if (mine && member<VARLEN>(p, it, qt, j)) {
+                if (s_iss > 0) {
+                  ok = mbar_wait(&s_free[t], (s_iss - 1) & 1, w);
+                  if (!ok) break;
+                  tc_fence_after();
+                }
+                issue_s(t, ks);
+                ++s_iss;
+              }
+              tc_commit(&kv_empty[ks]);
+              if (jn >= e) tc_commit(&q_empty);  // the item's last QK^T
+            }
+            if (jp >= 0) {
+              const uint32_t vi = kv_iter - 1, vs = vi % C::NSLOT;  // V of key tile jp
+              ok = mbar_wait(&kv_full[vs], (vi / C::NSLOT) & 1, w);
+              if (!ok) break;
+              tc_fence_after();
+              if (mine && member<VARLEN>(p, it, qt, jp)) {
+                ok = mbar_wait(&p_full[t], pv_iss & 1, w);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(t, vs, first_pv ? 0u : 1u);
+                tc_commit(&pv_done[t]);
+                first_pv = false;
+                ++pv_iss;
+              }
+              tc_commit(&kv_empty[vs]);
+            }
+            if (j < e) kv_iter += 2;
+            jp = j < e ? j : -1;
+            j = jn;
+          }
+          if (!ok) break;
+        }
+      } else {
       for (;; ++item_iter) {
         int idx;
         ok = take_item(item_iter, idx);
@@ -327,6 +417,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = t_lo; t < t_hi && t < tiles; ++t) tc_commit(&o_full[t]);
         if (!q_released) tc_commit(&q_empty);
       }
+      }
       if (issued) {
         // Every MMA issued by this thread must be finished before tensor
         // memory is released.
@@ -337,16 +428,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
   } else {
-    regs_inc<208>();  // may only raise them
+    regs_inc<C::REG_SMX>();  // may only raise them
     // ------------------------------------------------------------ softmax
     const int t = (warp - 4) >> 2;         // query tile of this warpgroup
     const int quarter = warp & 3;          // tensor-memory lane quarter
     const int r = quarter * 32 + lane;     // row within the tile
     const uint32_t lane_bits = uint32_t(quarter * 32) << 16;
     const uint32_t t_s = tmem + lane_bits + t * 128;
-    const uint32_t t_o = tmem + lane_bits + 256 + t * D;
+    const uint32_t t_o = tmem + lane_bits + C::COL_O + t * D;
+    const uint32_t t_p = tmem + lane_bits + C::COL_P + t * 64;  // SPLIT_P
     const float sl2 = p.scale_log2;
     uint32_t s_cnt = 0, o_cnt = 0;
+    uint32_t np = 0;  // P tiles written so far (SPLIT_P)
     bool ok = true;
 
     for (uint32_t k = 0;; ++k) {
@@ -371,6 +464,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < BN; c += 32) FA_TMEM_LD_X32(t_s + c, (sraw + c));
         tc_wait_ld();
+        if constexpr (C::SPLIT_P) {
+          tc_fence_before();
+          mbar_arrive(&s_free[t]);  // the next QK^T may overwrite the scores
+        }
         float x[BN];
 #pragma unroll
         for (int c = 0; c < BN; ++c) x[c] = __uint_as_float(sraw[c]);
@@ -384,82 +481,154 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int c = 0; c < BN; ++c)
             if (c >= lim) x[c] = -INFINITY;
         }
-        // row max as eight independent chains, then a tree
-        float ma[8];
+        // Reference maximum m.  A row takes it from its scores when it has
+        // none yet (its first key tile, or every key so far masked); after
+        // that the exponentials use the reference they have, and only a key
+        // tile whose row sum reaches 2^16 (or is not finite) moves it: that
+        // tile is then redone on its own row maximum, and l and O are brought
+        // onto the new reference.  O / l does not depend on the reference.
+        auto row_max = [&]() {
+          float ma[8];  // eight independent chains, then a tree
 #pragma unroll
-        for (int k = 0; k < 8; ++k) ma[k] = x[k];
+          for (int k = 0; k < 8; ++k) ma[k] = x[k];
 #pragma unroll
-        for (int c = 8; c < BN; c += 8)
+          for (int c = 8; c < BN; c += 8)
 #pragma unroll
-          for (int k = 0; k < 8; ++k) ma[k] = fmaxf(ma[k], x[c + k]);
-        float mx = fmaxf(fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3])), fmaxf(fmaxf(ma[4], ma[5]), fmaxf(ma[6], ma[7])));
-        mx *= sl2;
-        const bool grow = mx > m + RESCALE_THRESHOLD;
-        float alpha = 1.0f;
-        if (grow) {
-          alpha = ex2_approx(m - mx);  // 0 when m == -inf
-          m = mx;
-          l *= alpha;
-        }
-        if (__any_sync(0xffffffffu, grow && !first)) {
-          // The reference maximum moved for some row of this warp: bring its
-          // O accumulator onto the new reference (rows that did not move
-          // multiply by 1).  Before the first PV of an item there is nothing
-          // to rescale: that PV overwrites O.
-          const float a = (grow && !first) ? alpha : 1.0f;
+            for (int k = 0; k < 8; ++k) ma[k] = fmaxf(ma[k], x[c + k]);
+          return sl2 * fmaxf(fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3])),
+                             fmaxf(fmaxf(ma[4], ma[5]), fmaxf(ma[6], ma[7])));
+        };
+        // P = 2^(x sl2 - m) as bf16 into tensor memory (over the scores, or
+        // into P's own columns); returns the row sum of this key tile.
+        const uint32_t t_pw = C::SPLIT_P ? t_p : t_s;
+        auto exp_pass = [&]() {
+          const float m_use = (m == -INFINITY) ? 0.0f : m;  // a row with no key yet: P = 0
+          float rsa[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // row sum, eight chains
 #pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t v[32];
-            FA_TMEM_LD_X32(t_o + c, v);
-            tc_wait_ld();
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pk[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
-            FA_TMEM_ST_X32(t_o + c, v);
+            for (int i = 0; i < 32; ++i) {
+              const float p0 = ex2_approx(fmaf(x[64 * h + 2 * i], sl2, -m_use));
+              const float p1 = ex2_approx(fmaf(x[64 * h + 2 * i + 1], sl2, -m_use));
+              rsa[(2 * i) & 7] += p0;
+              rsa[(2 * i + 1) & 7] += p1;
+              pk[i] = pack_bf16x2(p0, p1);
+            }
+            FA_TMEM_ST_X32(t_pw + 32 * h, pk);
           }
+          return ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
+        };
+        const bool need_m = m == -INFINITY;
+        if (__any_sync(0xffffffffu, need_m)) {
+          const float mx = row_max();
+          if (need_m) m = mx;  // l and O are still zero for such a row
+        }
+        if constexpr (C::SPLIT_P) {
+          if (np > 0) {
+            // The previous PV has finished: it no longer reads P's columns,
+            // and O holds every product so far (for a rescale below).
+            ok = mbar_wait_warp(&pv_done[t], (np - 1) & 1, w);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          ++np;
+        }
+        float rs = exp_pass();
+        const bool redo = !(rs < 65536.0f);
+        if (__any_sync(0xffffffffu, redo)) {
+          float a = 1.0f;
+          if (redo) {
+            const float mx = row_max();  // >= m + 9 here, since rs >= 2^16
+            a = ex2_approx(m - mx);
+            m = mx;
+            l *= a;
+          }
+          // Bring O onto the new reference (rows that kept theirs multiply by
+          // 1).  Before the item's first PV there is nothing to rescale: that
+          // PV overwrites O.
+          if (!first) {
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+              uint32_t v[32];
+              FA_TMEM_LD_X32(t_o + c, v);
+              tc_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
+              FA_TMEM_ST_X32(t_o + c, v);
+            }
+          }
+          tc_wait_st();
+          rs = exp_pass();
         }
         first = false;
-        const float m_use = (m == -INFINITY) ? 0.0f : m;
-        float rsa[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // row sum, eight chains
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float p0 = ex2_approx(fmaf(x[64 * h + 2 * i], sl2, -m_use));
-            const float p1 = ex2_approx(fmaf(x[64 * h + 2 * i + 1], sl2, -m_use));
-            rsa[(2 * i) & 7] += p0;
-            rsa[(2 * i + 1) & 7] += p1;
-            pk[i] = pack_bf16x2(p0, p1);
-          }
-          FA_TMEM_ST_X32(t_s + 32 * h, pk);
-        }
-        l += ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
+        l += rs;
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[t]);
       }
       if (!ok) break;
       // ---- epilogue: O / l and LSE
-      ok = mbar_wait_warp(&o_full[t], o_cnt & 1, w);
+      if constexpr (C::SPLIT_P) {
+        // the tile's last PV (none if no key tile reached the tile: then
+        // l = 0 and O is written as zeros)
+        if (!first) ok = mbar_wait_warp(&pv_done[t], (np - 1) & 1, w);
+      } else {
+        ok = mbar_wait_warp(&o_full[t], o_cnt & 1, w);
+        ++o_cnt;
+      }
       if (!ok) break;
-      ++o_cnt;
       tc_fence_after();
       const bool live = l > 0.0f && row < it.Lq;  // false for a row that sees no key, or padding
       const float inv_l = live ? 1.0f / l : 0.0f;
       __nv_bfloat16* orow = p.O + ((size_t)it.bh * p.N + row) * D;
+      if constexpr (C::OSTAGE_BYTES > 0) {
+        // Lane i puts row i of the warp's 32 (128 bytes: eight 16-byte
+        // chunks, chunk k at slot k ^ (i & 7), so that eight lanes cover all
+        // banks), then each store instruction writes four whole rows.
+        uint8_t* ws = sO + (warp - 4) * 32 * D * 2;
+        __syncwarp();  // every lane has read the previous item's rows
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        uint32_t v[32];
-        FA_TMEM_LD_X32(t_o + c, v);
-        tc_wait_ld();
-        uint32_t pk[16];
+        for (int c = 0; c < D; c += 32) {
+          uint32_t v[32];
+          FA_TMEM_LD_X32(t_o + c, v);
+          tc_wait_ld();
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = live ? pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l) : 0u;
-        if (row < p.N && FA_IN_BOUNDS(p.status, ((size_t)it.bh * p.N + row) * D + c, 32, (size_t)p.BH * p.N * D)) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+          for (int i = 0; i < 16; ++i)
+            pk[i] = live ? pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l) : 0u;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) {
+            const int k = c / 8 + i;
+            *reinterpret_cast<uint4*>(ws + lane * 128 + ((k ^ (lane & 7)) * 16)) =
+                make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+        __syncwarp();
+        const int row0 = qt * BM + quarter * 32;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int ci = k * 32 + lane, rr = ci >> 3, ch = ci & 7;
+          const uint4 val = *reinterpret_cast<const uint4*>(ws + rr * 128 + ((ch ^ (rr & 7)) * 16));
+          const int grow = row0 + rr;
+          if (grow < p.N && FA_IN_BOUNDS(p.status, ((size_t)it.bh * p.N + grow) * D + ch * 8, 8, (size_t)p.BH * p.N * D))
+            *reinterpret_cast<uint4*>(p.O + ((size_t)it.bh * p.N + grow) * D + ch * 8) = val;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t v[32];
+          FA_TMEM_LD_X32(t_o + c, v);
+          tc_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = live ? pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l) : 0u;
+          if (row < p.N && FA_IN_BOUNDS(p.status, ((size_t)it.bh * p.N + row) * D + c, 32, (size_t)p.BH * p.N * D)) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
         }
       }
       if (row < p.N && FA_IN_BOUNDS(p.status, (size_t)it.bh * p.N + row, 1, (size_t)p.BH * p.N))
