@@ -191,7 +191,13 @@ struct Cfg {
   // The dynamic region starts 1024-byte aligned (the extern declaration
   // asks for it), so no slack is added: at d = 128 this is 226 KB, which
   // with the static barriers fills the 227 KB a CTA may use.
-  static constexpr int SMEM_BYTES = OFF_LD + NST * 1024;
+  // d = 64: each softmax warp stages its 32 rows of dV, then of dK (its 32
+  // of the 64 columns, bf16: 2 KB) so that they leave eight rows per store
+  // instruction.  (At d = 128 shared memory is full; there an item spans
+  // many query tiles and its epilogue matters little.)
+  static constexpr int OFF_EPI = OFF_LD + NST * 1024;
+  static constexpr int EPI_BYTES = D == 64 ? 8 * 32 * 64 : 0;
+  static constexpr int SMEM_BYTES = OFF_EPI + EPI_BYTES;
   // Tensor memory columns.  S^T fp32 in [0,128); once read, P^T (bf16) goes
   // to [0,64).  dP^T fp32 in [128,256); once read, dS^T (bf16) goes to
   // [128,192).  The score columns are thus free as soon as dV has been
@@ -705,19 +711,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float mul = g == 0 ? 1.0f : p.scale;
         __nv_bfloat16* dst = (g == 0 ? p.dV : p.dK) + gbase;
         const int colbase = (g == 0 ? C::COL_DV : C::COL_DK) + hf * (D / 2);
-#pragma unroll
-        for (int c = 0; c < D / 2; c += 32) {
+        if constexpr (C::EPI_BYTES > 0) {
+          // Lane i puts its 64 bytes (four 16-byte chunks, chunk c at slot
+          // c ^ ((i >> 1) & 3): eight lanes cover all banks) into the warp's
+          // 2 KB; then lanes 4r..4r+3 write row r of each group of eight.
+          uint8_t* ws = smem + C::OFF_EPI + (warp - 4) * 2048;
           uint32_t v[32];
-          FA_TMEM_LD_X32(tmem + lane_bits + colbase + c, v);
+          FA_TMEM_LD_X32(tmem + lane_bits + colbase, v);
           tc_wait_ld();
-          uint32_t pk[16];
+          __syncwarp();  // the warp has read out what it staged before
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = any ? pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul) : 0u;
-          if (store && FA_IN_BOUNDS(p.status, gbase + hf * (D / 2) + c, 32, (size_t)p.BH * p.Nk * D)) {
-            uint4* o = reinterpret_cast<uint4*>(dst + hf * (D / 2) + c);
+          for (int c = 0; c < 4; ++c) {
+            uint32_t q[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) o[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            for (int e = 0; e < 4; ++e)
+              q[e] = any ? pack_bf16x2(__uint_as_float(v[8 * c + 2 * e]) * mul, __uint_as_float(v[8 * c + 2 * e + 1]) * mul)
+                         : 0u;
+            *reinterpret_cast<uint4*>(ws + lane * 64 + ((c ^ ((lane >> 1) & 3)) * 16)) = make_uint4(q[0], q[1], q[2], q[3]);
+          }
+          __syncwarp();
+          const int key0 = it.j * BK + quarter * 32;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int rr = 8 * k + (lane >> 2), cc = lane & 3;
+            const uint4 val = *reinterpret_cast<const uint4*>(ws + rr * 64 + ((cc ^ ((rr >> 1) & 3)) * 16));
+            const size_t e0 = ((size_t)it.bh * p.Nk + key0 + rr) * D + hf * 32 + cc * 8;
+            if (key0 + rr < p.Nk && FA_IN_BOUNDS(p.status, e0, 8, (size_t)p.BH * p.Nk * D))
+              *reinterpret_cast<uint4*>((g == 0 ? p.dV : p.dK) + e0) = val;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < D / 2; c += 32) {
+            uint32_t v[32];
+            FA_TMEM_LD_X32(tmem + lane_bits + colbase + c, v);
+            tc_wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              pk[e] = any ? pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul) : 0u;
+            if (store && FA_IN_BOUNDS(p.status, gbase + hf * (D / 2) + c, 32, (size_t)p.BH * p.Nk * D)) {
+              uint4* o = reinterpret_cast<uint4*>(dst + hf * (D / 2) + c);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) o[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            }
           }
         }
       }
