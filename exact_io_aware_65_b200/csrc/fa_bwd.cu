@@ -31,8 +31,9 @@
 // CTA roles (512 threads): warp 0 TMA producer; warp 1 MMA issuer; warps
 // 4..11 softmax (thread = key row; warps 4..7 take query columns 0..63,
 // warps 8..11 columns 64..127); warps 12..15 dQ drain (thread = query row).
-// Tensor memory: S^T [0,128), then P^T (bf16) in [0,64); dP^T [128,256),
-// then dS^T (bf16) in [128,192); dV [256, 256+d); dK [256+d, 256+2d).  The
+// Tensor memory: S^T [0,128), then P^T (bf16) in [0,32) and [64,96); dP^T
+// [128,256), then dS^T (bf16) in [128,160) and [192,224); dV [256, 256+d);
+// dK [256+d, 256+2d).  The
 // MMA order per query tile is dV, next S^T, dK, dQ, next dP^T, so the
 // softmax of the next tile overlaps three products.  The dQ tile reuses the
 // dP^T columns for d = 128 (the next dP^T waits for the drain) and has two
@@ -198,11 +199,17 @@ struct Cfg {
   static constexpr int OFF_EPI = OFF_LD + NST * 1024;
   static constexpr int EPI_BYTES = D == 64 ? 8 * 32 * 64 : 0;
   static constexpr int SMEM_BYTES = OFF_EPI + EPI_BYTES;
-  // Tensor memory columns.  S^T fp32 in [0,128); once read, P^T (bf16) goes
-  // to [0,64).  dP^T fp32 in [128,256); once read, dS^T (bf16) goes to
-  // [128,192).  The score columns are thus free as soon as dV has been
-  // issued, so the next tile's S^T can follow it directly.
+  // Tensor memory columns.  S^T fp32 in [0,128); once read, P^T (bf16
+  // pairs) goes to [0,32) and [64,96): each column half of the softmax packs
+  // its 64 queries into the first 32 of its own 64 score columns, so neither
+  // half writes where the other is still reading.  Likewise dP^T fp32 in
+  // [128,256), then dS^T in [128,160) and [192,224).  The score columns are
+  // free as soon as dV has been issued, so the next tile's S^T can follow it
+  // directly.
   static constexpr int COL_S = 0, COL_P = 0, COL_DP = 128, COL_DS = 128;
+  // Column of the s-th 16-query slice (K = 16 of a gradient product) of
+  // packed P^T or dS^T starting at `base`.
+  __host__ __device__ static constexpr uint32_t col_packed(int base, int s) { return base + (s >> 2) * 64 + (s & 3) * 8; }
   static constexpr int COL_DV = 256, COL_DK = 256 + D;
   // dQ: d = 128 reuses the dP^T columns once dK has read dS^T (one buffer,
   // so the next dP^T waits for the drain); d = 64 has two spare 64-column
@@ -278,11 +285,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
 
   __shared__ __align__(8) uint64_t kv_full, kv_empty, s_full, dp_full, p_full, ds_full, dkdv_full, mma_drain;
-  // The two column halves of a lane quarter write packed bf16 results into
-  // columns the other half may still be reading as fp32 scores: each half
-  // arrives once its score loads are done and waits for the other before
-  // storing.
-  __shared__ __align__(8) uint64_t s_read, dp_read;
   // The dQ drain stages a tile in shared memory, in one or two parts, before
   // each bulk reduce-add (dq_staged[h]: all 128 drain threads have written
   // part h; dq_half: the first part has been read out).  One barrier per
@@ -318,8 +320,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(&ds_full, 256);
     mbar_init(&dkdv_full, 1);
     mbar_init(&mma_drain, 1);
-    mbar_init(&s_read, 256);
-    mbar_init(&dp_read, 256);
     mbar_init(&dq_staged[0], 128);
     mbar_init(&dq_staged[1], 128);
     mbar_init(&dq_half, 1);
@@ -525,7 +525,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
 #pragma unroll
           for (int s = 0; s < BQ / 16; ++s)
-            mma_ts(tmem + C::COL_DV, tmem + C::COL_P + s * 8, desc_at(gdO, s * 2048), IDESC_G,
+            mma_ts(tmem + C::COL_DV, tmem + C::col_packed(C::COL_P, s), desc_at(gdO, s * 2048), IDESC_G,
                    (n > 0 || s > 0) ? 1u : 0u);
           // S^T of the next query tile goes in now: its columns were last read
           // by the dV product just issued, and its softmax can then overlap
@@ -543,7 +543,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
 #pragma unroll
           for (int s = 0; s < BQ / 16; ++s)
-            mma_ts(tmem + C::COL_DK, tmem + C::COL_DS + s * 8, desc_at(gQ, s * 2048), IDESC_G,
+            mma_ts(tmem + C::COL_DK, tmem + C::col_packed(C::COL_DS, s), desc_at(gQ, s * 2048), IDESC_G,
                    (n > 0 || s > 0) ? 1u : 0u);
           const uint32_t b = dq_iter % C::NDQ;
           if (D == 64 && dq_iter >= (uint32_t)C::NDQ) {
@@ -618,8 +618,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           FA_TMEM_LD_X32(tmem + lane_bits + C::COL_S + hf * 64, sr);
           FA_TMEM_LD_X32(tmem + lane_bits + C::COL_S + hf * 64 + 32, (sr + 32));
           tc_wait_ld();
-          tc_fence_before();
-          mbar_arrive(&s_read);
           const float4* l4 = reinterpret_cast<const float4*>(sL);
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
@@ -637,10 +635,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             pk[2 * u + 1] = pack_bf16x2(pv[2], pv[3]);
           }
         }
-        ok = mbar_wait_warp(&s_read, par, w);
-        if (!ok) break;
-        tc_fence_after();
-        FA_TMEM_ST_X32(tmem + lane_bits + C::COL_P + hf * 32, pk);
+        // over the first 32 of this half's own 64 score columns, all loaded
+        FA_TMEM_ST_X32(tmem + lane_bits + C::COL_P + hf * 64, pk);
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full);
@@ -654,10 +650,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t dr[32];
           FA_TMEM_LD_X32(tmem + lane_bits + C::COL_DP + hf * 64 + cc * 32, dr);
           tc_wait_ld();
-          if (cc == 1) {
-            tc_fence_before();
-            mbar_arrive(&dp_read);
-          }
           const float4* d4 = reinterpret_cast<const float4*>(sD + cc * 32);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -671,12 +663,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             dk[cc * 16 + u * 2 + 1] = pack_bf16x2(g2, g3);
           }
         }
-        // dS^T overwrites dP^T columns the other column half may still be
-        // reading: wait until both halves have loaded theirs.
-        ok = mbar_wait_warp(&dp_read, par, w);
-        if (!ok) break;
-        tc_fence_after();
-        FA_TMEM_ST_X32(tmem + lane_bits + C::COL_DS + hf * 32, dk);
+        // over the first 32 of this half's own 64 dP^T columns, all loaded
+        FA_TMEM_ST_X32(tmem + lane_bits + C::COL_DS + hf * 64, dk);
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(&ds_full);  // dK may start
