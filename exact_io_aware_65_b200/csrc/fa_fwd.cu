@@ -69,9 +69,10 @@ struct Cfg {
   static constexpr int CHUNKS = D / 64;          // 64-column (128-byte) chunks per row
   static constexpr int CHUNK_BYTES = BN * 128;   // one chunk of a tile
   static constexpr int NSLOT = D == 64 ? 8 : 4;  // K/V ring slots
-  // d = 64: each softmax warp stages its 32 rows of O (bf16) here so that
-  // they go out to global memory four whole rows per store instruction.
-  static constexpr int OSTAGE_BYTES = D == 64 ? 8 * 32 * D * 2 : 0;
+  // Each softmax warp stages 64 columns of its 32 rows of O (bf16, 4 KB) at
+  // a time here, so that they go out four whole 128-byte row pieces per
+  // store instruction.
+  static constexpr int OSTAGE_BYTES = 8 * 32 * 128;
   static constexpr int SMEM_BYTES = 2 * TILE_BYTES + NSLOT * TILE_BYTES + OSTAGE_BYTES + 1024;
   // MMA issuer threads.  Issuing blocks while the tensor core's queue is
   // full, so with one issuer a tile's PV can wait behind the other tile's
@@ -581,53 +582,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const bool live = l > 0.0f && row < it.Lq;  // false for a row that sees no key, or padding
       const float inv_l = live ? 1.0f / l : 0.0f;
-      __nv_bfloat16* orow = p.O + ((size_t)it.bh * p.N + row) * D;
-      if constexpr (C::OSTAGE_BYTES > 0) {
-        // Lane i puts row i of the warp's 32 (128 bytes: eight 16-byte
-        // chunks, chunk k at slot k ^ (i & 7), so that eight lanes cover all
-        // banks), then each store instruction writes four whole rows.
-        uint8_t* ws = sO + (warp - 4) * 32 * D * 2;
-        __syncwarp();  // every lane has read the previous item's rows
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t v[32];
-          FA_TMEM_LD_X32(t_o + c, v);
-          tc_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = live ? pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l) : 0u;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int k = c / 8 + i;
-            *reinterpret_cast<uint4*>(ws + lane * 128 + ((k ^ (lane & 7)) * 16)) =
-                make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          }
-        }
-        __syncwarp();
+      {
+        // Per 64 columns: lane i puts row i of the warp's 32 (128 bytes:
+        // eight 16-byte chunks, chunk k at slot k ^ (i & 7), so that eight
+        // lanes cover all banks), then each store instruction writes four
+        // rows' 128 bytes.
+        uint8_t* ws = sO + (warp - 4) * 4096;
         const int row0 = qt * BM + quarter * 32;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int ci = k * 32 + lane, rr = ci >> 3, ch = ci & 7;
-          const uint4 val = *reinterpret_cast<const uint4*>(ws + rr * 128 + ((ch ^ (rr & 7)) * 16));
-          const int grow = row0 + rr;
-          if (grow < p.N && FA_IN_BOUNDS(p.status, ((size_t)it.bh * p.N + grow) * D + ch * 8, 8, (size_t)p.BH * p.N * D))
-            *reinterpret_cast<uint4*>(p.O + ((size_t)it.bh * p.N + grow) * D + ch * 8) = val;
-        }
-      } else {
+        for (int g = 0; g < D / 64; ++g) {
+          __syncwarp();  // every lane has read what the warp staged before
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t v[32];
-          FA_TMEM_LD_X32(t_o + c, v);
-          tc_wait_ld();
-          uint32_t pk[16];
+          for (int c = 0; c < 64; c += 32) {
+            uint32_t v[32];
+            FA_TMEM_LD_X32(t_o + 64 * g + c, v);
+            tc_wait_ld();
+            uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = live ? pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l) : 0u;
-          if (row < p.N && FA_IN_BOUNDS(p.status, ((size_t)it.bh * p.N + row) * D + c, 32, (size_t)p.BH * p.N * D)) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+            for (int i = 0; i < 16; ++i)
+              pk[i] = live ? pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l) : 0u;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            for (int i = 0; i < 4; ++i) {
+              const int k = c / 8 + i;
+              *reinterpret_cast<uint4*>(ws + lane * 128 + ((k ^ (lane & 7)) * 16)) =
+                  make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+          }
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int ci = k * 32 + lane, rr = ci >> 3, ch = ci & 7;
+            const uint4 val = *reinterpret_cast<const uint4*>(ws + rr * 128 + ((ch ^ (rr & 7)) * 16));
+            const int grow = row0 + rr;
+            const size_t e0 = ((size_t)it.bh * p.N + grow) * D + 64 * g + ch * 8;
+            if (grow < p.N && FA_IN_BOUNDS(p.status, e0, 8, (size_t)p.BH * p.N * D))
+              *reinterpret_cast<uint4*>(p.O + e0) = val;
           }
         }
       }
