@@ -455,8 +455,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       float l = 0.0f;
       bool first = true;  // no PV has written this tile's O yet
       const int e = kv_end<VARLEN>(p, it);
-      for (int j = next_union<VARLEN>(p, it, 0); j < e; j = next_union<VARLEN>(p, it, j + 1)) {
-        if (!member<VARLEN>(p, it, qt, j)) continue;
+      // The key tiles this query tile visits, in order.  Under a block mask
+      // the warp reads its row of the mask 32 key tiles at a time (one byte a
+      // lane, then a ballot) instead of one dependent load per key tile.
+      uint32_t mbits = 0;
+      int mbase = -64;  // first key tile of the 32 in mbits
+      auto next_key = [&](int j) -> int {
+        if (p.mask_kind != FA_MASK_BLOCK) {
+          while (j < e && !member<VARLEN>(p, it, qt, j)) ++j;
+          return j < e ? j : e;
+        }
+        while (j < e) {
+          if (j < mbase || j >= mbase + 32) {
+            mbase = j & ~31;
+            const int jj = mbase + lane;
+            mbits = __ballot_sync(0xffffffffu, jj < e && member<VARLEN>(p, it, qt, jj));
+          }
+          const uint32_t rest = mbits >> (j - mbase);
+          if (rest) return j + __ffs(rest) - 1;
+          j = mbase + 32;
+        }
+        return e;
+      };
+      for (int j = next_key(0); j < e; j = next_key(j + 1)) {
         ok = mbar_wait_warp(&s_full[t], s_cnt & 1, w);
         if (!ok) break;
         ++s_cnt;
