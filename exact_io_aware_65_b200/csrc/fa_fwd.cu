@@ -63,17 +63,28 @@ __device__ uint32_t g_claim[SCHED_SLOTS];  // dynamic claims so far
 __device__ uint32_t g_done[SCHED_SLOTS];   // CTAs that stopped claiming
 constexpr float LN2 = 0.69314718055994530942f;
 
-template <int D>
+template <int D, int PIPES>
 struct Cfg {
   static constexpr int TILE_BYTES = BN * D * 2;  // one Q, K or V tile
   static constexpr int CHUNKS = D / 64;          // 64-column (128-byte) chunks per row
   static constexpr int CHUNK_BYTES = BN * 128;   // one chunk of a tile
-  static constexpr int NSLOT = D == 64 ? 8 : 4;  // K/V ring slots
+  // PIPES = 2 (d = 64 under a block mask): two independent pipelines per
+  // CTA.  Each has its own producer warp (0, 3), MMA issuer (1, 2), softmax
+  // warpgroup (4..7, 8..11), Q tile, K/V ring and stream of work items, one
+  // query tile each; they share only the CTA's shared and tensor memory, so
+  // one pipeline's softmax, item change or load wait overlaps the other's
+  // work, and neither loads key tiles only the other needs.  PIPES = 1: one
+  // pipeline, work items of two query tiles sharing one K/V stream (better
+  // where the two tiles need the same key tiles: no mask, causal).
+  static_assert(PIPES == 1 || (PIPES == 2 && D == 64), "two pipelines need the d = 64 column plan");
+  static constexpr bool DUAL = PIPES == 2;
+  static constexpr int NPIPE = PIPES;
+  static constexpr int NSLOT = DUAL ? 4 : (D == 64 ? 8 : 4);  // K/V ring slots per pipeline
   // Each softmax warp stages 64 columns of its 32 rows of O (bf16, 4 KB) at
   // a time here, so that they go out four whole 128-byte row pieces per
   // store instruction.
   static constexpr int OSTAGE_BYTES = 8 * 32 * 128;
-  static constexpr int SMEM_BYTES = 2 * TILE_BYTES + NSLOT * TILE_BYTES + OSTAGE_BYTES + 1024;
+  static constexpr int SMEM_BYTES = 2 * TILE_BYTES + NPIPE * NSLOT * TILE_BYTES + OSTAGE_BYTES + 1024;
   // MMA issuer threads.  Issuing blocks while the tensor core's queue is
   // full, so with one issuer a tile's PV can wait behind the other tile's
   // products.  d = 64: one issuer per query tile (short products, so the
@@ -85,7 +96,9 @@ struct Cfg {
   static constexpr bool SPLIT_P = D == 64;
   static constexpr uint32_t COL_P = 256;                   // + 64 t (SPLIT_P)
   static constexpr uint32_t COL_O = SPLIT_P ? 384 : 256;   // + d t
-  static constexpr int CONSUMERS = ISSUERS + 8;  // of the item ring: issuers + softmax warps
+  // Consumers of a pipeline's item ring: its issuer(s) and softmax warps.
+  static constexpr int CONSUMERS = DUAL ? 1 + 4 : ISSUERS + 8;
+  static constexpr int PIPE_ISSUERS = DUAL ? 1 : ISSUERS;  // commits per Q / K/V release
   // Registers per thread after the split (launch: 168): producer and issuer
   // warpgroup, then each softmax warpgroup.  The d = 64 softmax holds a
   // whole score row and spills below 224.
@@ -96,24 +109,25 @@ struct Cfg {
 
 // VARLEN: per-sequence lengths are read (else every sequence has N, Nk and
 // the sizes stay compile-time-free of extra registers).
-template <int D, bool VARLEN>
+template <int D, bool VARLEN, int PIPES>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                const __grid_constant__ CUtensorMap mapV, const Params p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, PIPES>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                        // 2 tiles
-  uint8_t* sKV = smem + 2 * C::TILE_BYTES;   // NSLOT tiles
-  uint8_t* sO = sKV + C::NSLOT * C::TILE_BYTES;  // OSTAGE_BYTES
+  uint8_t* sQ = smem;                        // 2 tiles (DUAL: pipeline q's at q)
+  uint8_t* sKV = smem + 2 * C::TILE_BYTES;   // NPIPE rings of NSLOT tiles
+  uint8_t* sO = sKV + C::NPIPE * C::NSLOT * C::TILE_BYTES;  // OSTAGE_BYTES
 
-  __shared__ __align__(8) uint64_t q_full, q_empty, mma_drain[2];
-  __shared__ __align__(8) uint64_t kv_full[C::NSLOT], kv_empty[C::NSLOT];
+  // Per pipeline: Q, K/V ring, item ring.
+  __shared__ __align__(8) uint64_t q_full[2], q_empty[2], mma_drain[2];
+  __shared__ __align__(8) uint64_t kv_full[2][C::NSLOT], kv_empty[2][C::NSLOT];
   __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_full[2];
   __shared__ __align__(8) uint64_t s_free[2], pv_done[2];  // SPLIT_P only
-  // The producer claims work items and passes them to the other roles.
-  __shared__ __align__(8) uint64_t item_full[RING], item_empty[RING];
-  __shared__ int item_ring[RING];
+  // A pipeline's producer claims work items and passes them to its other roles.
+  __shared__ __align__(8) uint64_t item_full[2][RING], item_empty[2][RING];
+  __shared__ int item_ring[2][RING];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -121,13 +135,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    mbar_init(&q_full, 1);
-    mbar_init(&q_empty, C::ISSUERS);  // one commit from each MMA issuer
     mbar_init(&mma_drain[0], 1);
     mbar_init(&mma_drain[1], 1);
-    for (int i = 0; i < C::NSLOT; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], C::ISSUERS);
+    for (int q = 0; q < C::NPIPE; ++q) {
+      mbar_init(&q_full[q], 1);
+      mbar_init(&q_empty[q], C::PIPE_ISSUERS);  // one commit from each of its MMA issuers
+      for (int i = 0; i < C::NSLOT; ++i) {
+        mbar_init(&kv_full[q][i], 1);
+        mbar_init(&kv_empty[q][i], C::PIPE_ISSUERS);
+      }
+      for (int r = 0; r < RING; ++r) {
+        mbar_init(&item_full[q][r], 1);
+        mbar_init(&item_empty[q][r], C::CONSUMERS);
+      }
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
@@ -136,17 +156,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&s_free[t], BM);
       mbar_init(&pv_done[t], 1);
     }
-    for (int r = 0; r < RING; ++r) {
-      mbar_init(&item_full[r], 1);
-      mbar_init(&item_empty[r], C::CONSUMERS);
-    }
     fence_barrier_init();
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) {
+  if ((warp == 0 || (C::DUAL && warp == 3)) && lane == 0) {
     tma_prefetch_desc(&mapQ);
     tma_prefetch_desc(&mapK);
     tma_prefetch_desc(&mapV);
@@ -158,19 +174,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = tmem_base_sh;
   const WaitCtx w{p.timeout_ns, &abort_flag, p.status};
 
-  auto take_item = [&](uint32_t k, int& idx) -> bool {
+  auto take_item = [&](int q, uint32_t k, int& idx) -> bool {
     const uint32_t slot = k % RING;
-    if (!mbar_wait(&item_full[slot], (k / RING) & 1, w)) return false;
-    idx = *reinterpret_cast<volatile int*>(&item_ring[slot]);
-    mbar_arrive(&item_empty[slot]);
+    if (!mbar_wait(&item_full[q][slot], (k / RING) & 1, w)) return false;
+    idx = *reinterpret_cast<volatile int*>(&item_ring[q][slot]);
+    mbar_arrive(&item_empty[q][slot]);
     return true;
   };
-  auto take_item_warp = [&](uint32_t k, int& idx) -> bool {
+  auto take_item_warp = [&](int q, uint32_t k, int& idx) -> bool {
     const uint32_t slot = k % RING;
-    if (!mbar_wait_warp(&item_full[slot], (k / RING) & 1, w)) return false;
-    idx = *reinterpret_cast<volatile int*>(&item_ring[slot]);
+    if (!mbar_wait_warp(&item_full[q][slot], (k / RING) & 1, w)) return false;
+    idx = *reinterpret_cast<volatile int*>(&item_ring[q][slot]);
     __syncwarp();
-    if (lane == 0) mbar_arrive(&item_empty[slot]);
+    if (lane == 0) mbar_arrive(&item_empty[q][slot]);
     return true;
   };
 
@@ -180,52 +196,61 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // the launch total).
   if (warp < 4) {
     regs_dec<C::REG_CTL>();  // may only lower the 168 registers of the launch
-  if (warp == 0) {
+  if (warp == 0 || (C::DUAL && warp == 3)) {
     // ------------------------------------------------------------ producer
+    // (of pipeline q)
     if (lane == 0) {
+      const int q = warp == 0 ? 0 : 1;
       uint32_t kv_iter = 0, item_iter = 0;
+      bool q_loading = false;  // this item's Q load was issued
       bool ok = true;
       for (;; ++item_iter) {
         const uint32_t slot = item_iter % RING;
-        ok = mbar_wait(&item_empty[slot], ((item_iter / RING) & 1) ^ 1, w);
+        ok = mbar_wait(&item_empty[q][slot], ((item_iter / RING) & 1) ^ 1, w);
         if (!ok) break;
-        int idx = item_iter == 0 ? (int)blockIdx.x : (int)gridDim.x + (int)atomicAdd(&g_claim[p.slot], 1u);
+        // Pipeline q of CTA b starts on item NPIPE b + q, then claims items
+        // NPIPE gridDim.x, NPIPE gridDim.x + 1, ...
+        int idx = item_iter == 0 ? (int)(blockIdx.x * C::NPIPE) + q
+                                 : (int)(gridDim.x * C::NPIPE) + (int)atomicAdd(&g_claim[p.slot], 1u);
         if (idx > p.n_items) idx = p.n_items;
-        item_ring[slot] = idx;
-        mbar_arrive(&item_full[slot]);
+        item_ring[q][slot] = idx;
+        mbar_arrive(&item_full[q][slot]);
         if (idx >= p.n_items) break;
         const Item it = item_at<VARLEN>(p, idx);
-        ok = mbar_wait(&q_empty, (item_iter & 1) ^ 1, w);
+        q_loading = false;
+        ok = mbar_wait(&q_empty[q], (item_iter & 1) ^ 1, w);
         if (!ok) break;
-        mbar_arrive_expect_tx(&q_full, C::TILE_BYTES * (it.has1 ? 2 : 1));
+        mbar_arrive_expect_tx(&q_full[q], C::TILE_BYTES * (it.has1 ? 2 : 1));
 #pragma unroll
         for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_3d(sQ + c * C::CHUNK_BYTES, &mapQ, &q_full, c * 64, it.q0 * BM, it.bh);
+          tma_load_3d(sQ + q * C::TILE_BYTES + c * C::CHUNK_BYTES, &mapQ, &q_full[q], c * 64, it.q0 * BM, it.bh);
         if (it.has1) {
 #pragma unroll
           for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_3d(sQ + C::TILE_BYTES + c * C::CHUNK_BYTES, &mapQ, &q_full, c * 64, it.q1 * BM, it.bh);
+            tma_load_3d(sQ + C::TILE_BYTES + c * C::CHUNK_BYTES, &mapQ, &q_full[q], c * 64, it.q1 * BM, it.bh);
         }
+        q_loading = true;
         const int e = kv_end<VARLEN>(p, it);
         for (int j = next_union<VARLEN>(p, it, 0); ok && j < e; j = next_union<VARLEN>(p, it, j + 1)) {
           for (int kv = 0; kv < 2; ++kv) {
             const uint32_t slot = kv_iter % C::NSLOT;
-            ok = mbar_wait(&kv_empty[slot], ((kv_iter / C::NSLOT) & 1) ^ 1, w);
+            ok = mbar_wait(&kv_empty[q][slot], ((kv_iter / C::NSLOT) & 1) ^ 1, w);
             if (!ok) break;
-            mbar_arrive_expect_tx(&kv_full[slot], C::TILE_BYTES);
-            uint8_t* dst = sKV + slot * C::TILE_BYTES;
+            mbar_arrive_expect_tx(&kv_full[q][slot], C::TILE_BYTES);
+            uint8_t* dst = sKV + (q * C::NSLOT + slot) * C::TILE_BYTES;
             const CUtensorMap* m = kv == 0 ? &mapK : &mapV;
 #pragma unroll
             for (int c = 0; c < C::CHUNKS; ++c)
-              tma_load_3d(dst + c * C::CHUNK_BYTES, m, &kv_full[slot], c * 64, j * BN, it.bh);
+              tma_load_3d(dst + c * C::CHUNK_BYTES, m, &kv_full[q][slot], c * 64, j * BN, it.bh);
             ++kv_iter;
           }
         }
         if (!ok) break;
       }
-      // This CTA claims no more (its last claim ran past the end, or it
-      // aborted); the last CTA to get here resets the counter slot.
-      if (atomicAdd(&g_done[p.slot], 1u) == gridDim.x - 1) {
+      // This pipeline claims no more (its last claim ran past the end, or it
+      // aborted); the last pipeline of the launch to get here resets the
+      // counter slot.
+      if (atomicAdd(&g_done[p.slot], 1u) == gridDim.x * C::NPIPE - 1) {
         g_claim[p.slot] = 0u;
         g_done[p.slot] = 0u;
       }
@@ -236,9 +261,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t n = kv_iter < (uint32_t)C::NSLOT ? kv_iter : (uint32_t)C::NSLOT;
         for (uint32_t i = 0; i < n; ++i) {
           const uint32_t k = kv_iter - 1 - i;
-          mbar_drain_wait(&kv_full[k % C::NSLOT], (k / C::NSLOT) & 1, dl);
+          mbar_drain_wait(&kv_full[q][k % C::NSLOT], (k / C::NSLOT) & 1, dl);
         }
-        if (item_iter > 0) mbar_drain_wait(&q_full, (item_iter - 1) & 1, dl);
+        // the last Q load issued: this item's, or the previous item's
+        const uint32_t last_q = q_loading ? item_iter : item_iter - 1;
+        if (q_loading || item_iter > 0) mbar_drain_wait(&q_full[q], last_q & 1, dl);
       }
     }
   } else if (warp == 1 || (C::ISSUERS == 2 && warp == 2)) {
@@ -285,32 +312,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
 
       if constexpr (C::SPLIT_P) {
-        // One tile per issuer.  Per union key step j (K of j at ring index
-        // kv_iter, its V at kv_iter + 1): S = Q K_j^T once the softmax has
-        // read the previous scores, then O += P V for the key tile before j
-        // once its P is written.  Every S, P and PV is counted over the whole
-        // launch, so the n-th of each pairs with the n-th arrival.
+        // The issuer of query tile t: with two pipelines the one tile of
+        // pipeline t's items, else tile t of the pipeline's pairs.  Per key
+        // step j (K of j at ring index kv_iter, its V at kv_iter + 1):
+        // S = Q K_j^T once the softmax has read the previous scores, then
+        // O += P V for the key tile before j once its P is written.  Every
+        // S, P and PV is counted over the whole launch, so the n-th of each
+        // pairs with the n-th arrival.
         const int t = warp - 1;
+        const int q = C::DUAL ? t : 0;         // pipeline
+        const uint32_t ring0 = q * C::NSLOT;  // its first ring slot
         uint32_t s_iss = 0, pv_iss = 0;
         for (;; ++item_iter) {
           int idx;
-          ok = take_item(item_iter, idx);
+          ok = take_item(q, item_iter, idx);
           if (!ok || idx >= p.n_items) break;
           const Item it = item_at<VARLEN>(p, idx);
-          const bool mine = t == 0 || it.has1;
-          const int qt = t == 0 ? it.q0 : it.q1;
-          ok = mbar_wait(&q_full, item_iter & 1, w);
+          const bool mine = C::DUAL || t == 0 || it.has1;
+          const int qt = (C::DUAL || t == 0) ? it.q0 : it.q1;
+          ok = mbar_wait(&q_full[q], item_iter & 1, w);
           if (!ok) break;
           tc_fence_after();
           const int e = kv_end<VARLEN>(p, it);
           int j = next_union<VARLEN>(p, it, 0), jp = -1;
-          if (j >= e) tc_commit(&q_empty);  // no key tile: Q was not read
+          if (j >= e) tc_commit(&q_empty[q]);  // no key tile: Q was not read
           bool first_pv = true;
           while (ok && (j < e || jp >= 0)) {
             const int jn = j < e ? next_union<VARLEN>(p, it, j + 1) : e;
             if (j < e) {
               const uint32_t ks = kv_iter % C::NSLOT;
-              ok = mbar_wait(&kv_full[ks], (kv_iter / C::NSLOT) & 1, w);
+              ok = mbar_wait(&kv_full[q][ks], (kv_iter / C::NSLOT) & 1, w);
               if (!ok) break;
               tc_fence_after();
               if (mine && member<VARLEN>(p, it, qt, j)) {
@@ -319,27 +350,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   if (!ok) break;
                   tc_fence_after();
                 }
-                issue_s(t, ks);
+                issue_s(t, ring0 + ks);
                 ++s_iss;
               }
-              tc_commit(&kv_empty[ks]);
-              if (jn >= e) tc_commit(&q_empty);  // the item's last QK^T
+              tc_commit(&kv_empty[q][ks]);
+              if (jn >= e) tc_commit(&q_empty[q]);  // the item's last QK^T
             }
             if (jp >= 0) {
               const uint32_t vi = kv_iter - 1, vs = vi % C::NSLOT;  // V of key tile jp
-              ok = mbar_wait(&kv_full[vs], (vi / C::NSLOT) & 1, w);
+              ok = mbar_wait(&kv_full[q][vs], (vi / C::NSLOT) & 1, w);
               if (!ok) break;
               tc_fence_after();
               if (mine && member<VARLEN>(p, it, qt, jp)) {
                 ok = mbar_wait(&p_full[t], pv_iss & 1, w);
                 if (!ok) break;
                 tc_fence_after();
-                issue_pv(t, vs, first_pv ? 0u : 1u);
+                issue_pv(t, ring0 + vs, first_pv ? 0u : 1u);
                 tc_commit(&pv_done[t]);
                 first_pv = false;
                 ++pv_iss;
               }
-              tc_commit(&kv_empty[vs]);
+              tc_commit(&kv_empty[q][vs]);
             }
             if (j < e) kv_iter += 2;
             jp = j < e ? j : -1;
@@ -350,11 +381,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else {
       for (;; ++item_iter) {
         int idx;
-        ok = take_item(item_iter, idx);
+        ok = take_item(0, item_iter, idx);
         if (!ok || idx >= p.n_items) break;
         const Item it = item_at<VARLEN>(p, idx);
         const int tiles = it.has1 ? 2 : 1;  // tiles [0, tiles) exist
-        ok = mbar_wait(&q_full, item_iter & 1, w);
+        ok = mbar_wait(&q_full[0], item_iter & 1, w);
         if (!ok) break;
         tc_fence_after();
         const int e = kv_end<VARLEN>(p, it);
@@ -367,15 +398,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         bool q_released = false;
         if (j < e) {
           const uint32_t ks = kv_iter % C::NSLOT;
-          ok = mbar_wait(&kv_full[ks], (kv_iter / C::NSLOT) & 1, w);
+          ok = mbar_wait(&kv_full[0][ks], (kv_iter / C::NSLOT) & 1, w);
           if (!ok) break;
           tc_fence_after();
           for (int t = t_lo; t < t_hi && t < tiles; ++t)
             if (member<VARLEN>(p, it, t == 0 ? it.q0 : it.q1, j)) issue_s(t, ks);
-          tc_commit(&kv_empty[ks]);
+          tc_commit(&kv_empty[0][ks]);
           ++kv_iter;
           if (jn >= e) {
-            tc_commit(&q_empty);
+            tc_commit(&q_empty[0]);
             q_released = true;
           }
         }
@@ -383,8 +414,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int jnn = jn < e ? next_union<VARLEN>(p, it, jn + 1) : e;
           const uint32_t vs = kv_iter % C::NSLOT;
           const uint32_t ksn = (kv_iter + 1) % C::NSLOT;
-          ok = mbar_wait(&kv_full[vs], (kv_iter / C::NSLOT) & 1, w);
-          if (ok && jn < e) ok = mbar_wait(&kv_full[ksn], ((kv_iter + 1) / C::NSLOT) & 1, w);
+          ok = mbar_wait(&kv_full[0][vs], (kv_iter / C::NSLOT) & 1, w);
+          if (ok && jn < e) ok = mbar_wait(&kv_full[0][ksn], ((kv_iter + 1) / C::NSLOT) & 1, w);
           if (!ok) break;
           tc_fence_after();
           for (int t = t_lo; t < t_hi && t < tiles && ok; ++t) {
@@ -400,12 +431,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (jn < e && member<VARLEN>(p, it, qt, jn)) issue_s(t, ksn);
           }
           if (!ok) break;
-          tc_commit(&kv_empty[vs]);
+          tc_commit(&kv_empty[0][vs]);
           if (jn < e) {
-            tc_commit(&kv_empty[ksn]);
+            tc_commit(&kv_empty[0][ksn]);
             kv_iter += 2;
             if (!q_released && jnn >= e) {
-              tc_commit(&q_empty);
+              tc_commit(&q_empty[0]);
               q_released = true;
             }
           } else {
@@ -416,7 +447,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (!ok) break;
         for (int t = t_lo; t < t_hi && t < tiles; ++t) tc_commit(&o_full[t]);
-        if (!q_released) tc_commit(&q_empty);
+        if (!q_released) tc_commit(&q_empty[0]);
       }
       }
       if (issued) {
@@ -445,11 +476,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     for (uint32_t k = 0;; ++k) {
       int idx;
-      ok = take_item_warp(k, idx);
+      ok = take_item_warp(C::DUAL ? t : 0, k, idx);
       if (!ok || idx >= p.n_items) break;
       const Item it = item_at<VARLEN>(p, idx);
-      if (t == 1 && !it.has1) continue;
-      const int qt = t == 0 ? it.q0 : it.q1;
+      if (!C::DUAL && t == 1 && !it.has1) continue;
+      const int qt = (C::DUAL || t == 0) ? it.q0 : it.q1;  // DUAL: each pipeline's item is one tile
       const int row = qt * BM + r;
       float m = -INFINITY;  // reference maximum, scaled log2 units
       float l = 0.0f;
@@ -676,7 +707,10 @@ fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void
   p.H = pr.H;
   p.seqlens_q = pr.seqlens_q;
   p.seqlens_k = pr.seqlens_k;
-  p.n_pairs = (pr.nq + 1) / 2;
+  // d = 64 under a block mask: two pipelines of one-tile items
+  const bool dual = pr.d == 64 && pr.mask_kind == FA_MASK_BLOCK;
+  p.tiles_per_item = dual ? 1 : 2;
+  p.n_pairs = (pr.nq + p.tiles_per_item - 1) / p.tiles_per_item;
   p.n_items = p.n_pairs * pr.BH;
   p.group = pr.BH < 8 ? pr.BH : 8;
   p.mask_kind = pr.mask_kind;
@@ -688,7 +722,9 @@ fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void
   p.status = st;
   static std::atomic<uint32_t> next_slot{0};
   p.slot = next_slot.fetch_add(1u, std::memory_order_relaxed) % fwd::SCHED_SLOTS;
-  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  const int npipe = dual ? 2 : 1;
+  const int want = (p.n_items + npipe - 1) / npipe;  // CTAs that get a first item in every pipeline
+  const int grid = want < num_sms() ? want : num_sms();
   auto run = [&](auto kern, int smem) -> bool {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return false;
     kern<<<grid, fwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, p);
@@ -696,12 +732,15 @@ fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void
   };
   const bool varlen = pr.seqlens_q || pr.seqlens_k;
   bool ok;
-  if (pr.d == 64)
-    ok = varlen ? run(fwd::fwd_kernel<64, true>, fwd::Cfg<64>::SMEM_BYTES)
-                : run(fwd::fwd_kernel<64, false>, fwd::Cfg<64>::SMEM_BYTES);
+  if (pr.d == 64 && dual)
+    ok = varlen ? run(fwd::fwd_kernel<64, true, 2>, fwd::Cfg<64, 2>::SMEM_BYTES)
+                : run(fwd::fwd_kernel<64, false, 2>, fwd::Cfg<64, 2>::SMEM_BYTES);
+  else if (pr.d == 64)
+    ok = varlen ? run(fwd::fwd_kernel<64, true, 1>, fwd::Cfg<64, 1>::SMEM_BYTES)
+                : run(fwd::fwd_kernel<64, false, 1>, fwd::Cfg<64, 1>::SMEM_BYTES);
   else
-    ok = varlen ? run(fwd::fwd_kernel<128, true>, fwd::Cfg<128>::SMEM_BYTES)
-                : run(fwd::fwd_kernel<128, false>, fwd::Cfg<128>::SMEM_BYTES);
+    ok = varlen ? run(fwd::fwd_kernel<128, true, 1>, fwd::Cfg<128, 1>::SMEM_BYTES)
+                : run(fwd::fwd_kernel<128, false, 1>, fwd::Cfg<128, 1>::SMEM_BYTES);
   if (!ok) return FA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

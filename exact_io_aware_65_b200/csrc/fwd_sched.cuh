@@ -19,6 +19,9 @@ constexpr int BN = 128;              // keys per tile
 
 struct Params {
   int BH, N, nq, n_pairs, n_items, mask_kind;  // N, nq: query rows and tiles
+  // Query tiles per work item: 2 (a pair, n_pairs = ceil(nq / 2)) or 1
+  // (n_pairs = nq: one tile per item).
+  int tiles_per_item;
   int Nk, nk, off;  // key rows and tiles; causal: query i sees keys j <= i + off
   int H;            // heads per batch element (a head's batch element is bh / H)
   // Optional per-batch-element lengths (device int [B], nullptr: N and Nk):
@@ -41,7 +44,7 @@ struct Item {
   int Lq, Lk, off, nkb;  // this sequence's query rows and keys, causal offset, key tiles
 };
 
-// Work item idx -> (head, pair of query tiles).  Heads are taken in groups
+// Work item idx -> (head, pair of query tiles, or one query tile).  Heads are taken in groups
 // of p.group so that the K/V tiles in flight belong to a few heads and stay
 // in L2; within a group later query tiles come first, so that under a causal
 // mask the longest items start earliest (and, claimed dynamically, the short
@@ -54,9 +57,9 @@ __host__ __device__ __forceinline__ Item item_at(const Params& p, int idx) {
   const int gsize = min(p.group, p.BH - g * p.group);
   const int c = p.n_pairs - 1 - r / gsize;
   it.bh = g * p.group + r % gsize;
-  it.q0 = 2 * c;
-  it.q1 = 2 * c + 1;
-  it.has1 = it.q1 < p.nq;
+  it.q0 = p.tiles_per_item * c;
+  it.q1 = it.q0 + 1;
+  it.has1 = p.tiles_per_item == 2 && it.q1 < p.nq;
   if (VARLEN) {
     const int b = it.bh / p.H;
     const bool bok = FA_IN_BOUNDS(p.status, b, 1, p.BH / p.H);

@@ -64,14 +64,15 @@ void fail(const char* what, const Problem& pr, int a, int b, int c) {
 }
 
 template <bool VARLEN>
-void check_fwd(const Problem& pr) {
+void check_fwd(const Problem& pr, int tiles_per_item) {
   using namespace fa::fwd;
   Params p = {};
+  p.tiles_per_item = tiles_per_item;
   const int BH = pr.B * pr.H;
   p.BH = BH; p.N = pr.Nq; p.nq = pr.nq(); p.Nk = pr.Nk; p.nk = pr.nk(); p.off = pr.Nk - pr.Nq; p.H = pr.H;
   p.seqlens_q = VARLEN ? pr.lq.data() : nullptr;
   p.seqlens_k = VARLEN ? pr.lk.data() : nullptr;
-  p.n_pairs = (p.nq + 1) / 2;
+  p.n_pairs = (p.nq + tiles_per_item - 1) / tiles_per_item;
   p.n_items = p.n_pairs * BH;
   p.group = BH < 8 ? BH : 8;
   p.mask_kind = pr.kind;
@@ -185,10 +186,12 @@ int main() {
                   pr.lq.push_back(u == 0 ? 0 : u == 1 ? pr.Nq : (int)(rnd() % (pr.Nq + 1)));
                   pr.lk.push_back(u == 0 ? pr.Nk : u == 1 ? pr.Nk : (int)(rnd() % (pr.Nk + 1)));
                 }
-                check_fwd<true>(pr);
+                check_fwd<true>(pr, 2);
+                check_fwd<true>(pr, 1);
                 check_bwd<true>(pr);
               } else {
-                check_fwd<false>(pr);
+                check_fwd<false>(pr, 2);
+                check_fwd<false>(pr, 1);
                 check_bwd<false>(pr);
               }
               ++cases;

@@ -40,6 +40,7 @@ MUTANTS = [
      "return min(qt * BM + BM - 2, it.Lq - 1) + it.off;"),
     ("bwd_add_rank", "bwd_sched.cuh", "  return (uint32_t)j;", "  return (uint32_t)(j > 0 ? j - 1 : 0);"),
     ("bwd_item_map", "bwd_sched.cuh", "  it.j = r / gsize;", "  it.j = r % gsize;"),
+    ("fwd_single_tile_items", "fwd_sched.cuh", "  it.q0 = p.tiles_per_item * c;", "  it.q0 = 2 * c;"),
 ]
 
 
