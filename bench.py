@@ -44,7 +44,8 @@ DEFAULT_WORKLOAD = "long_s8k_d128_causal"
 # The two-sequence variant (a 1 GiB cache, still far above L2) is the one
 # profiled with ncu.
 DECODE_WORKLOADS = {"decode_b8_h32_kv32k_d128": dict(B=8, H=32, Nq=1, Nk=32768, d=128, mask="causal"),
-                    "decode_b2_h32_kv32k_d128": dict(B=2, H=32, Nq=1, Nk=32768, d=128, mask="causal")}
+                    "decode_b2_h32_kv32k_d128": dict(B=2, H=32, Nq=1, Nk=32768, d=128, mask="causal"),
+                    "decode_b8_h32_q16_kv32k_d128": dict(B=8, H=32, Nq=16, Nk=32768, d=128, mask="causal")}
 DECODE_METRIC = "decode attention: K/V cache bytes streamed per second (bf16), % of measured HBM bandwidth"
 
 L2_BYTES = 126 * 2 ** 20

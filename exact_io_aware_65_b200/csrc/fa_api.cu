@@ -208,6 +208,10 @@ fa_status fa_bwd_stage(int stage, const void* Q, const void* K, const void* V, c
                     workspace_bytes, stream);
 }
 
+// fa_decode hands problems with at least this many queries per head (and at
+// least one head per SM) to the tensor-core forward.
+constexpr int DECODE_TC_MIN_NQ = 4;
+
 size_t fa_decode_workspace_size(int B, int H, int Nq, int Nk, int d) {
   if (B <= 0 || H <= 0 || Nq <= 0 || Nq > 16 || Nk <= 0 || (d != 64 && d != 128)) return 0;
   const long long bh = (long long)B * H;
@@ -226,6 +230,11 @@ fa_status fa_decode(const void* Q, const void* K, const void* V, int B, int H, i
   const size_t need = decode_workspace_bytes(p.BH, Nq, Nk, d);
   if (need == 0) return FA_ERR_CUDA;
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FA_ERR_WORKSPACE;
+  // With several queries per head and a head for every SM, the tensor-core
+  // forward (one work item per head, the cache read once per head) fills the
+  // GPU and outruns the split-key kernel, whose per-query work runs on the
+  // CUDA cores.
+  if (Nq >= DECODE_TC_MIN_NQ && p.BH >= num_sms()) return launch_fwd(p, Q, K, V, O, LSE, (cudaStream_t)stream);
   return launch_decode(p, Q, K, V, O, LSE, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 

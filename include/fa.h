@@ -178,7 +178,11 @@ fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, 
  * KV cache), forward only.  The same exact attention as fa_fwd_qk, computed
  * by splitting the keys across the GPU and merging the partial softmax
  * results by their running maxima and sums (log-sum-exp); meant for the
- * shapes where fa_fwd_qk would leave most of the GPU idle.
+ * shapes where fa_fwd_qk would leave most of the GPU idle.  With Nq >= 4
+ * and at least as many heads (B H) as the GPU has SMs, the call runs the
+ * tensor-core forward of fa_fwd_qk instead (one work item per head), which
+ * then fills the GPU and reads the cache once per head at a higher rate;
+ * the workspace is still required and goes unused.
  * In:  Q [B,H,Nq,d] bf16 with 1 <= Nq <= 16; K, V [B,H,Nk,d] bf16, Nk >= 1;
  *      mask_kind FA_MASK_NONE or FA_MASK_CAUSAL (bottom-right aligned as in
  *      fa_fwd_qk: query i sees keys j <= i + (Nk - Nq)); scale > 0;

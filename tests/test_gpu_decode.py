@@ -51,6 +51,22 @@ def test_decode_agrees_with_tensor_core_forward(case):
     assert (L1 - L2).abs().max().item() <= 1e-3
 
 
+@pytest.mark.parametrize("case", [(4, 40, 8, 2048, 128, "causal"), (2, 80, 16, 1000, 64, "none"),
+                                  (1, 160, 4, 300, 64, "causal")])
+def test_decode_with_a_head_per_sm_matches_oracle(case):
+    # four or more queries and at least one head per SM (148): the call runs
+    # the tensor-core forward; the result must be the same attention
+    B, H, Nq, Nk, d, m = case
+    scale = float(np.float32(d ** -0.5))
+    x = workloads.make_cross_inputs(B, H, Nq, Nk, d, m, seed=Nq + Nk)
+    dv = to_dev(x)
+    O, L = fa.decode(dv["Q"], dv["K"], dv["V"], m, scale)
+    assert fa.device_status() == 0
+    Or, Lr = oracle.fwd(x["Q"], x["K"], x["V"], m, None, scale)
+    assert_o(f64(O), Or, str(case))
+    assert_lse(f64(L), Lr, str(case))
+
+
 def test_decode_refuses_what_it_does_not_do():
     q = torch.zeros((1, 1, 17, 64), dtype=torch.bfloat16, device="cuda")
     k = torch.zeros((1, 1, 100, 64), dtype=torch.bfloat16, device="cuda")
