@@ -16,8 +16,12 @@
 //   warps 4..7    softmax for query tile 0; warps 8..11 for query tile 1.
 //                 Thread r owns query row r: it reads its score row from
 //                 tensor memory, keeps the row max m and row sum l in
-//                 registers, writes P (bf16) back over the scores, and does
+//                 registers, writes P (bf16) into tensor memory, and does
 //                 the final O / l and LSE epilogue.
+// At d = 64 under a block mask the CTA runs two independent pipelines
+// (Cfg::DUAL): warps 0 and 3 produce, 1 and 2 issue, 4..7 and 8..11 do the
+// softmax, each pipeline with its own Q tile, K/V ring and work items of one
+// query tile.
 // Tensor memory (512 columns):
 //   d = 128: S/P of tile t at [128 t, 128 t + 128) (P, bf16, over the scores),
 //            O of tile t at [256 + 128 t, 384 + 128 t).  A tile's next QK^T
