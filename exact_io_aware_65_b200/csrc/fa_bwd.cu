@@ -229,10 +229,11 @@ struct Cfg {
   static_assert(DQ_SLOT_OFF + DQ_PART_BYTES <= 2 * TILE_BYTES, "dQ part exceeds its stage");
   // Registers per thread of the producer/MMA, softmax and drain warpgroups
   // (setmaxnreg).  Launch: 512 threads x 128; 128 x (REG_CTL + 2 REG_SMX +
-  // REG_DRN) must stay <= 65536.  Chosen so that ptxas spills nothing (d=128)
-  // or next to nothing (d=64).
-  static constexpr uint32_t REG_CTL = D == 128 ? 104 : 88;
-  static constexpr uint32_t REG_SMX = D == 128 ? 128 : 136;
+  // REG_DRN) must stay <= 65536.  ptxas spills nothing at either d; at
+  // d = 128, 136 for the softmax rather than 128 took the main kernel from
+  // 1.294 to 1.283 ms.
+  static constexpr uint32_t REG_CTL = 88;
+  static constexpr uint32_t REG_SMX = 136;
   static constexpr uint32_t REG_DRN = 152;
   static_assert(REG_CTL + 2 * REG_SMX + REG_DRN <= 512, "register split exceeds the launch");
   // setmaxnreg.dec may only lower and setmaxnreg.inc only raise the 128
