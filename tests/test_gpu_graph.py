@@ -26,18 +26,23 @@ def _inputs(B, H, N, d, mask, seed):
 
 
 def _step(st, w, deterministic):
-    O, L = fa.fwd(st["Q"], st["K"], st["V"], w.mask, None, w.scale, O=st["O"], LSE=st["LSE"])
-    fa.bwd(st["Q"], st["K"], st["V"], O, st["dO"], L, w.mask, None, w.scale, dQ=st["dQ"], dK=st["dK"],
+    m = st.get("mask")
+    O, L = fa.fwd(st["Q"], st["K"], st["V"], w.mask, m, w.scale, O=st["O"], LSE=st["LSE"])
+    fa.bwd(st["Q"], st["K"], st["V"], O, st["dO"], L, w.mask, m, w.scale, dQ=st["dQ"], dK=st["dK"],
            dV=st["dV"], workspace=st["ws"], deterministic=deterministic)
 
 
 @pytest.mark.parametrize("deterministic", [False, True], ids=["atomic-dq", "ordered-dq"])
-@pytest.mark.parametrize("shape", [(2, 3, 700, 64, "causal"), (1, 4, 1100, 128, "none")],
+# (the block-mask case runs the d = 64 forward's two-pipeline kernel, whose
+# work counter is reset by the last of its 2 x grid pipelines)
+@pytest.mark.parametrize("shape", [(2, 3, 700, 64, "causal"), (1, 4, 1100, 128, "none"), (2, 3, 900, 64, "block")],
                          ids=lambda s: "x".join(map(str, s)))
 def test_fwd_bwd_graph_replays_equal_eager(shape, deterministic):
     B, H, N, d, mask = shape
     w, x0 = _inputs(B, H, N, d, mask, seed=11)
     st = {k: x0[k].cuda() for k in ("Q", "K", "V", "dO")}
+    if x0["mask"] is not None:
+        st["mask"] = x0["mask"].cuda()
     st["O"] = torch.empty_like(st["Q"])
     st["LSE"] = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
     st["dQ"], st["dK"], st["dV"] = (torch.empty_like(st["Q"]) for _ in range(3))
@@ -60,6 +65,8 @@ def test_fwd_bwd_graph_replays_equal_eager(shape, deterministic):
         _, x = _inputs(B, H, N, d, mask, seed=100 + r)
         for k in ("Q", "K", "V", "dO"):
             st[k].copy_(x[k])
+        if x["mask"] is not None:
+            st["mask"].copy_(x["mask"])  # a new mask in the same buffer: read when the graph runs
         g.replay()
         got = {k: st[k].clone() for k in outs}
         assert fa.device_status() == 0
@@ -68,7 +75,7 @@ def test_fwd_bwd_graph_replays_equal_eager(shape, deterministic):
         exact = outs if deterministic else ("O", "LSE", "dK", "dV")
         for k in exact:
             assert torch.equal(got[k], st[k]), f"replay {r}: {k} differs from the eager call"
-        ref = oracle.bwd(x["Q"], x["K"], x["V"], x["dO"], mask, None, w.scale)
+        ref = oracle.bwd(x["Q"], x["K"], x["V"], x["dO"], mask, x["mask"], w.scale)
         assert_o(f64(got["O"]), ref["O"], f"replay {r}")
         assert_lse(f64(got["LSE"]), ref["LSE"], f"replay {r}")
         for k in ("dQ", "dK", "dV"):
