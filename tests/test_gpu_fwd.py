@@ -61,20 +61,21 @@ def test_fwd_block_mask_with_empty_rows():
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("mask", ["none", "causal"])
+@pytest.mark.parametrize("mask", ["none", "causal", "block"])
 @pytest.mark.parametrize("growth", [2.0, 0.5])
 def test_fwd_scores_growing_or_shrinking_along_the_keys(d, mask, growth):
     # K's key tile j is scaled by growth**j.  Growing: from the third key tile
     # on, each tile's exponentials outgrow the row's reference maximum by far
     # more than 2^16, so every such tile is redone on a new reference and O and
     # l are rescaled.  Shrinking: later tiles fall far below the reference.
+    # (The block mask at d = 64 runs the two-pipeline forward.)
     B, H, N = 1, 2, 768
     w = workloads.Workload("t", B, H, N, d, mask, float(np.float32(d ** -0.5)))
     x = workloads.make_inputs(w, 5, grad=False)
     f = torch.tensor([growth ** (j // 128) for j in range(N)], dtype=torch.float32)
     x["K"] = (x["K"].float() * f[None, None, :, None]).to(torch.bfloat16).contiguous()
     O, L = run_fwd(w, x)
-    Or, Lr = oracle.fwd(x["Q"], x["K"], x["V"], mask, None, w.scale)
+    Or, Lr = oracle.fwd(x["Q"], x["K"], x["V"], mask, x["mask"], w.scale)
     # Growing scores make each output row nearly one row of V (|O| up to ~4),
     # so the fixed absolute bound does not fit.  The bound here follows the
     # arithmetic: each weight of P is rounded to bf16 (relative error at most
@@ -82,7 +83,7 @@ def test_fwd_scores_growing_or_shrinking_along_the_keys(d, mask, growth):
     # 2^-8 sum_j w_ij |v_j| (w the exact softmax weights: the oracle's output
     # with |V| in place of V); rounding O to bf16 adds at most 2^-8 |O_i|; the
     # fp32 scores and the approximate exponential add far less than 1e-3.
-    Wabs, _ = oracle.fwd(x["Q"], x["K"], x["V"].abs(), mask, None, w.scale)
+    Wabs, _ = oracle.fwd(x["Q"], x["K"], x["V"].abs(), mask, x["mask"], w.scale)
     err = np.abs(f64(O) - Or)
     bound = 2.0 ** -8 * (Wabs + np.abs(Or)) + 1e-3
     assert (err <= bound).all(), f"growth {growth}: worst excess {(err - bound).max():.3e}"
