@@ -69,6 +69,20 @@ bool make_map_bf16(CUtensorMap* map, const void* base, int BH, int N, int d, int
   return r == CUDA_SUCCESS;
 }
 
+bool make_map_bf16_box(CUtensorMap* map, const void* base, int BH, int N, int d, int box_cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn || (box_cols != 32 && box_cols != 64)) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * (cuuint64_t)N};
+  cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  // the box's rows are 64 or 128 bytes: the swizzle of that width
+  const CUtensorMapSwizzle sw = box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_map_bf16_2d(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
   return make_map_bf16(map, base, 1, rows, cols, box_rows);
 }

@@ -281,6 +281,7 @@ template <int D, bool VARLEN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                 const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapdO,
+                const __grid_constant__ CUtensorMap mapdK, const __grid_constant__ CUtensorMap mapdV,
                 const Params p) {
   using C = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -702,13 +703,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int colbase = (g == 0 ? C::COL_DV : C::COL_DK) + hf * (D / 2);
         if constexpr (C::EPI_BYTES > 0) {
           // Lane i puts its 64 bytes (four 16-byte chunks, chunk c at slot
-          // c ^ ((i >> 1) & 3): eight lanes cover all banks) into the warp's
-          // 2 KB; then lanes 4r..4r+3 write row r of each group of eight.
+          // c ^ ((i >> 1) & 3), which is the 64-byte swizzle) into the warp's
+          // 2 KB; then lane 0 stores the 32 x 32 box with one tensor store
+          // (keys past Nk are not written).
           uint8_t* ws = smem + C::OFF_EPI + (warp - 4) * 2048;
           uint32_t v[32];
           FA_TMEM_LD_X32(tmem + lane_bits + colbase, v);
           tc_wait_ld();
-          __syncwarp();  // the warp has read out what it staged before
+          if (lane == 0) bulk_wait_read_all();  // the warp's previous store has read the buffer
+          __syncwarp();
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t q[4];
@@ -718,15 +721,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                          : 0u;
             *reinterpret_cast<uint4*>(ws + lane * 64 + ((c ^ ((lane >> 1) & 3)) * 16)) = make_uint4(q[0], q[1], q[2], q[3]);
           }
+          fence_proxy_async_smem();  // the generic-proxy writes, before the tensor store reads them
           __syncwarp();
-          const int key0 = it.j * BK + quarter * 32;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int rr = 8 * k + (lane >> 2), cc = lane & 3;
-            const uint4 val = *reinterpret_cast<const uint4*>(ws + rr * 64 + ((cc ^ ((rr >> 1) & 3)) * 16));
-            const size_t e0 = ((size_t)it.bh * p.Nk + key0 + rr) * D + hf * 32 + cc * 8;
-            if (key0 + rr < p.Nk && FA_IN_BOUNDS(p.status, e0, 8, (size_t)p.BH * p.Nk * D))
-              *reinterpret_cast<uint4*>((g == 0 ? p.dV : p.dK) + e0) = val;
+          if (lane == 0) {
+            tma_store_3d(g == 0 ? &mapdV : &mapdK, ws, hf * 32, it.j * BK + quarter * 32, it.bh);
+            bulk_commit_group();
           }
         } else {
 #pragma unroll
@@ -748,6 +747,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_before();
     }
+    if (C::EPI_BYTES > 0 && lane == 0) bulk_wait_all();  // this warp's dK/dV stores are done before the CTA leaves
   } else {
     regs_inc<C::REG_DRN>();
     // ------------------------------------------------------------ dQ drain
@@ -966,11 +966,15 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     p.dV = static_cast<__nv_bfloat16*>(dV);
     p.timeout_ns = wait_timeout_ns();
     p.status = st;
+    // dK and dV as 32 x 32 boxes for the d = 64 epilogue's tensor stores
+    CUtensorMap mdK, mdV;
+    if (!make_map_bf16_box(&mdK, dK, pr.BH, pr.Nk, pr.d, 32, 32) || !make_map_bf16_box(&mdV, dV, pr.BH, pr.Nk, pr.d, 32, 32))
+      return FA_ERR_CUDA;
     constexpr int smem = bwd::Cfg<D>::SMEM_BYTES;
     const int grid = p.n_items < sms ? p.n_items : sms;
     auto run = [&](auto kern) -> bool {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return false;
-      kern<<<grid, bwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, mdO, p);
+      kern<<<grid, bwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, mdO, mdK, mdV, p);
       return true;
     };
     const bool varlen = pr.seqlens_q || pr.seqlens_k;

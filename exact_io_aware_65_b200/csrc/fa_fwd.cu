@@ -116,7 +116,8 @@ struct Cfg {
 template <int D, bool VARLEN, int PIPES>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-               const __grid_constant__ CUtensorMap mapV, const Params p) {
+               const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapO,
+               const Params p) {
   using C = Cfg<D, PIPES>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -640,14 +641,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float inv_l = live ? 1.0f / l : 0.0f;
       {
         // Per 64 columns: lane i puts row i of the warp's 32 (128 bytes:
-        // eight 16-byte chunks, chunk k at slot k ^ (i & 7), so that eight
-        // lanes cover all banks), then each store instruction writes four
-        // rows' 128 bytes.
+        // eight 16-byte chunks, chunk k at slot k ^ (i & 7), which is the
+        // 128-byte swizzle), then lane 0 stores the 32 x 64 box with one
+        // tensor store (rows past N are not written).
         uint8_t* ws = sO + (warp - 4) * 4096;
         const int row0 = qt * BM + quarter * 32;
 #pragma unroll
         for (int g = 0; g < D / 64; ++g) {
-          __syncwarp();  // every lane has read what the warp staged before
+          if (lane == 0) bulk_wait_read_all();  // the warp's previous store has read the buffer
+          __syncwarp();
 #pragma unroll
           for (int c = 0; c < 64; c += 32) {
             uint32_t v[32];
@@ -664,15 +666,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
             }
           }
+          fence_proxy_async_smem();  // the generic-proxy writes, before the tensor store reads them
           __syncwarp();
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int ci = k * 32 + lane, rr = ci >> 3, ch = ci & 7;
-            const uint4 val = *reinterpret_cast<const uint4*>(ws + rr * 128 + ((ch ^ (rr & 7)) * 16));
-            const int grow = row0 + rr;
-            const size_t e0 = ((size_t)it.bh * p.N + grow) * D + 64 * g + ch * 8;
-            if (grow < p.N && FA_IN_BOUNDS(p.status, e0, 8, (size_t)p.BH * p.N * D))
-              *reinterpret_cast<uint4*>(p.O + e0) = val;
+          if (lane == 0) {
+            tma_store_3d(&mapO, ws, 64 * g, row0, it.bh);
+            bulk_commit_group();
           }
         }
       }
@@ -680,6 +678,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         p.LSE[(size_t)it.bh * p.N + row] = live ? (m + log2f(l)) * LN2 : -INFINITY;
       tc_fence_before();
     }
+    if (lane == 0) bulk_wait_all();  // this warp's O stores are done before the CTA leaves
   }
 
   tc_fence_before();
@@ -697,9 +696,9 @@ fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void
                      cudaStream_t s) {
   uint32_t* st = status_word();
   if (!st) return FA_ERR_CUDA;
-  CUtensorMap mQ, mK, mV;
+  CUtensorMap mQ, mK, mV, mO;
   if (!make_map_bf16(&mQ, Q, pr.BH, pr.N, pr.d, fwd::BM) || !make_map_bf16(&mK, K, pr.BH, pr.Nk, pr.d, fwd::BN) ||
-      !make_map_bf16(&mV, V, pr.BH, pr.Nk, pr.d, fwd::BN))
+      !make_map_bf16(&mV, V, pr.BH, pr.Nk, pr.d, fwd::BN) || !make_map_bf16_box(&mO, O, pr.BH, pr.N, pr.d, 64, 32))
     return FA_ERR_CUDA;
   fwd::Params p;
   p.BH = pr.BH;
@@ -731,7 +730,7 @@ fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void
   const int grid = want < num_sms() ? want : num_sms();
   auto run = [&](auto kern, int smem) -> bool {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return false;
-    kern<<<grid, fwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, p);
+    kern<<<grid, fwd::NUM_THREADS, smem, s>>>(mQ, mK, mV, mO, p);
     return true;
   };
   const bool varlen = pr.seqlens_q || pr.seqlens_k;

@@ -30,6 +30,9 @@ struct Problem {
 // dims (d, N, BH), box (64, box_rows, 1), 128-byte swizzle, zero fill out of
 // bounds.  Returns false on failure.
 bool make_map_bf16(CUtensorMap* map, const void* base, int BH, int N, int d, int box_rows);
+// The same [BH, N, d] view with a box of box_cols (32 or 64) x box_rows and the
+// swizzle of the box's row width (64 or 128 bytes): for tiled stores.
+bool make_map_bf16_box(CUtensorMap* map, const void* base, int BH, int N, int d, int box_cols, int box_rows);
 
 // Same for a 2-D row-major bf16 matrix [rows, cols] (used by the self-test).
 bool make_map_bf16_2d(CUtensorMap* map, const void* base, int rows, int cols, int box_rows);
