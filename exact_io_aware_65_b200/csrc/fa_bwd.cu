@@ -13,8 +13,9 @@
 //     dK_j  = scale sum_i dS_ij q_i,   dQ_i = scale sum_j dS_ij k_j
 //
 // Three kernels, all on the caller's stream:
-//   prep     D_i, LSE_i * log2(e) (padded to whole tiles) and a zeroed fp32
-//            dQ accumulator, in the workspace.
+//   prep     -D_i, -LSE_i * log2(e) (negated, so that the softmax adds them;
+//            padded to whole tiles) and a zeroed fp32 dQ accumulator, in the
+//            workspace.
 //   main     one persistent CTA per SM; a work item is one (head, 128-key
 //            tile).  K_j and V_j stay in shared memory, dK_j and dV_j
 //            accumulate in tensor memory across the query tiles that see
@@ -121,13 +122,13 @@ __global__ void __launch_bounds__(256) prep_kernel(const __nv_bfloat16* __restri
       if (li == 0) {
         if ((n & 127) == 0 && FA_IN_BOUNDS(status, (size_t)bh * (Npad / 128) + n / 128, 1, total / 128))
           turn[(size_t)bh * (Npad / 128) + n / 128] = 0u;
-        Dw[r] = acc;
+        Dw[r] = -acc;
         float l2 = INFINITY;  // padding rows and rows that saw no key: P = 0
         if (real && FA_IN_BOUNDS(status, (size_t)bh * N + n, 1, (size_t)BH * N)) {
           const float lse = LSE[(size_t)bh * N + n];
           if (lse > -INFINITY) l2 = lse * LOG2E;
         }
-        L2w[r] = l2;
+        L2w[r] = -l2;
       }
       float4* z = reinterpret_cast<float4*>(dq_acc + (size_t)r * D + li * 8);
       z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -620,14 +621,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           FA_TMEM_LD_X32(tmem + lane_bits + C::COL_S + hf * 64, sr);
           FA_TMEM_LD_X32(tmem + lane_bits + C::COL_S + hf * 64 + 32, (sr + 32));
           tc_wait_ld();
+          // (-LSE * log2e and -D are stored negated: two columns per packed
+          // fp32 instruction, each lane rounding as the scalar form)
           const float4* l4 = reinterpret_cast<const float4*>(sL);
+          const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             const float4 lv = l4[u];
-            float pv[4] = {ex2_approx(fmaf(__uint_as_float(sr[4 * u + 0]), sl2, -lv.x)),
-                           ex2_approx(fmaf(__uint_as_float(sr[4 * u + 1]), sl2, -lv.y)),
-                           ex2_approx(fmaf(__uint_as_float(sr[4 * u + 2]), sl2, -lv.z)),
-                           ex2_approx(fmaf(__uint_as_float(sr[4 * u + 3]), sl2, -lv.w))};
+            const float2 y0 = __ffma2_rn(make_float2(__uint_as_float(sr[4 * u + 0]), __uint_as_float(sr[4 * u + 1])),
+                                         sl2x2, make_float2(lv.x, lv.y));
+            const float2 y1 = __ffma2_rn(make_float2(__uint_as_float(sr[4 * u + 2]), __uint_as_float(sr[4 * u + 3])),
+                                         sl2x2, make_float2(lv.z, lv.w));
+            float pv[4] = {ex2_approx(y0.x), ex2_approx(y0.y), ex2_approx(y1.x), ex2_approx(y1.y)};
             if (masked) {
 #pragma unroll
               for (int e = 0; e < 4; ++e)
@@ -657,12 +662,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int u = 0; u < 8; ++u) {
             const float4 dv = d4[u];
             const uint32_t w0 = pk[cc * 16 + 2 * u], w1 = pk[cc * 16 + 2 * u + 1];
-            const float g0 = __uint_as_float(w0 << 16) * (__uint_as_float(dr[u * 4 + 0]) - dv.x);
-            const float g1 = __uint_as_float(w0 & 0xffff0000u) * (__uint_as_float(dr[u * 4 + 1]) - dv.y);
-            const float g2 = __uint_as_float(w1 << 16) * (__uint_as_float(dr[u * 4 + 2]) - dv.z);
-            const float g3 = __uint_as_float(w1 & 0xffff0000u) * (__uint_as_float(dr[u * 4 + 3]) - dv.w);
-            dk[cc * 16 + u * 2 + 0] = pack_bf16x2(g0, g1);
-            dk[cc * 16 + u * 2 + 1] = pack_bf16x2(g2, g3);
+            const float2 t0 = __fadd2_rn(make_float2(__uint_as_float(dr[u * 4 + 0]), __uint_as_float(dr[u * 4 + 1])),
+                                         make_float2(dv.x, dv.y));
+            const float2 t1 = __fadd2_rn(make_float2(__uint_as_float(dr[u * 4 + 2]), __uint_as_float(dr[u * 4 + 3])),
+                                         make_float2(dv.z, dv.w));
+            const float2 g01 = __fmul2_rn(make_float2(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xffff0000u)), t0);
+            const float2 g23 = __fmul2_rn(make_float2(__uint_as_float(w1 << 16), __uint_as_float(w1 & 0xffff0000u)), t1);
+            dk[cc * 16 + u * 2 + 0] = pack_bf16x2(g01.x, g01.y);
+            dk[cc * 16 + u * 2 + 1] = pack_bf16x2(g23.x, g23.y);
           }
         }
         // over the first 32 of this half's own 64 dP^T columns, all loaded
@@ -716,9 +723,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int c = 0; c < 4; ++c) {
             uint32_t q[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              q[e] = any ? pack_bf16x2(__uint_as_float(v[8 * c + 2 * e]) * mul, __uint_as_float(v[8 * c + 2 * e + 1]) * mul)
-                         : 0u;
+            for (int e = 0; e < 4; ++e) {
+              const float2 o = __fmul2_rn(make_float2(__uint_as_float(v[8 * c + 2 * e]), __uint_as_float(v[8 * c + 2 * e + 1])),
+                                          make_float2(mul, mul));
+              q[e] = any ? pack_bf16x2(o.x, o.y) : 0u;
+            }
             *reinterpret_cast<uint4*>(ws + lane * 64 + ((c ^ ((lane >> 1) & 3)) * 16)) = make_uint4(q[0], q[1], q[2], q[3]);
           }
           fence_proxy_async_smem();  // the generic-proxy writes, before the tensor store reads them
@@ -735,8 +744,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_wait_ld();
             uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              pk[e] = any ? pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul) : 0u;
+            for (int e = 0; e < 16; ++e) {
+              const float2 o = __fmul2_rn(make_float2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])),
+                                          make_float2(mul, mul));
+              pk[e] = any ? pack_bf16x2(o.x, o.y) : 0u;
+            }
             if (store && FA_IN_BOUNDS(p.status, gbase + hf * (D / 2) + c, 32, (size_t)p.BH * p.Nk * D)) {
               uint4* o = reinterpret_cast<uint4*>(dst + hf * (D / 2) + c);
 #pragma unroll

@@ -85,8 +85,8 @@ struct Cfg {
   static constexpr int NPIPE = PIPES;
   static constexpr int NSLOT = DUAL ? 4 : (D == 64 ? 8 : 4);  // K/V ring slots per pipeline
   // Each softmax warp stages 64 columns of its 32 rows of O (bf16, 4 KB) at
-  // a time here, so that they go out four whole 128-byte row pieces per
-  // store instruction.
+  // a time here, in the 128-byte swizzle, and writes them out with one
+  // tensor store.
   static constexpr int OSTAGE_BYTES = 8 * 32 * 128;
   static constexpr int SMEM_BYTES = 2 * TILE_BYTES + NPIPE * NSLOT * TILE_BYTES + OSTAGE_BYTES + 1024;
   // MMA issuer threads.  Issuing blocks while the tensor core's queue is
@@ -106,8 +106,8 @@ struct Cfg {
   // Registers per thread after the split (launch: 168): producer and issuer
   // warpgroup, then each softmax warpgroup.  The d = 64 softmax holds a
   // whole score row and spills below 224.
-  static constexpr int REG_CTL = D == 64 ? 56 : 88;
-  static constexpr int REG_SMX = D == 64 ? 224 : 208;
+  static constexpr int REG_CTL = D == 64 ? 56 : 72;
+  static constexpr int REG_SMX = D == 64 ? 224 : 216;
   static_assert(REG_CTL + 2 * REG_SMX <= 3 * 168, "register split exceeds the launch");
 };
 
@@ -561,21 +561,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t t_pw = C::SPLIT_P ? t_p : t_s;
         auto exp_pass = [&]() {
           const float m_use = (m == -INFINITY) ? 0.0f : m;  // a row with no key yet: P = 0
-          float rsa[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // row sum, eight chains
+          // Two columns per instruction (packed fp32 pairs) for the scaling
+          // and the row sum; each lane of a pair rounds as the scalar form.
+          const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(-m_use, -m_use);
+          float2 rsa[4] = {};  // row sum, eight chains in four pairs
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float p0 = ex2_approx(fmaf(x[64 * h + 2 * i], sl2, -m_use));
-              const float p1 = ex2_approx(fmaf(x[64 * h + 2 * i + 1], sl2, -m_use));
-              rsa[(2 * i) & 7] += p0;
-              rsa[(2 * i + 1) & 7] += p1;
-              pk[i] = pack_bf16x2(p0, p1);
+              const float2 y = __ffma2_rn(make_float2(x[64 * h + 2 * i], x[64 * h + 2 * i + 1]), sl2x2, nm2);
+              const float2 pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+              rsa[i & 3] = __fadd2_rn(rsa[i & 3], pp);
+              pk[i] = pack_bf16x2(pp.x, pp.y);
             }
             FA_TMEM_ST_X32(t_pw + 32 * h, pk);
           }
-          return ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
+          return ((rsa[0].x + rsa[0].y) + (rsa[1].x + rsa[1].y)) + ((rsa[2].x + rsa[2].y) + (rsa[3].x + rsa[3].y));
         };
         const bool need_m = m == -INFINITY;
         if (__any_sync(0xffffffffu, need_m)) {
@@ -657,8 +659,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_wait_ld();
             uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = live ? pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l) : 0u;
+            for (int i = 0; i < 16; ++i) {
+              const float2 o = __fmul2_rn(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])),
+                                          make_float2(inv_l, inv_l));
+              pk[i] = live ? pack_bf16x2(o.x, o.y) : 0u;
+            }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int k = c / 8 + i;
