@@ -187,7 +187,7 @@ struct Cfg {
   static constexpr int OFF_V = TILE_BYTES;
   static constexpr int OFF_DS = 2 * TILE_BYTES;           // dS^T, 128 x 128 bf16 (2 chunks)
   static constexpr int OFF_QD = 2 * TILE_BYTES + 32768;   // stages of (Q, dO)
-  // Per stage: the 128 LSE*log2(e) values then the 128 D values of the
+  // Per stage: the 128 -LSE*log2(e) values then the 128 -D values of the
   // stage's query tile (fp32, 1 KB).
   static constexpr int OFF_LD = OFF_QD + NST * 2 * TILE_BYTES;
   // The dynamic region starts 1024-byte aligned (the extern declaration
