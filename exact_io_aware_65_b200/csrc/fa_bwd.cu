@@ -680,7 +680,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // Shared-memory copy of dS^T (the A operand of dQ = dS K), 128-byte
         // swizzle: 16-byte unit u of row kr lives at unit (u ^ (kr & 7)).
         // With the split drain the buffer may still hold half of the
-        // previous dQ tile on its way to the accumulator.
+        // previous dQ tile on its way to the accumulator.  Otherwise its
+        // only other reader, the previous dQ product, has completed: the MMA
+        // warp issues this tile's dP^T after that product, and dp_full (the
+        // commit of both) was waited for above.
         if (D == 128 && !p.deterministic && s_cnt > 1) {
           ok = mbar_wait_warp(&sds_free, (s_cnt - 2) & 1, w);
           if (!ok) break;
