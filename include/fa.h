@@ -100,12 +100,13 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
 
 /* The three launches fa_bwd makes, callable one at a time with fa_bwd's
  * arguments (each call checks them the same way).  stage 0: prep -- the row
- * terms D_i = dO_i . O_i, LSE scaled to log2 units and a zeroed fp32 dQ
- * accumulator, all in the workspace; stage 1: main -- recompute P, produce dK
- * and dV, add dQ partial sums into the accumulator; stage 2: write
- * dQ = bf16(scale * accumulator).  fa_bwd(...) is exactly stages 0, 1, 2 in
- * order on one stream; a stage reads what the previous one left in the
- * workspace, so they must run in that order on the same workspace. */
+ * terms D_i = dO_i . O_i and LSE scaled to log2 units (both stored negated)
+ * and a zeroed fp32 dQ accumulator, all in the workspace; stage 1: main --
+ * recompute P, produce dK and dV, add dQ partial sums into the accumulator;
+ * stage 2: write dQ = bf16(scale * accumulator).  fa_bwd(...) is exactly
+ * stages 0, 1, 2 in order on one stream; a stage reads what the previous
+ * one left in the workspace, so they must run in that order on the same
+ * workspace. */
 fa_status fa_bwd_stage(int stage, const void* Q, const void* K, const void* V, const void* O,
                        const void* dO, const float* LSE, int B, int H, int N, int d, int mask_kind,
                        const uint8_t* block_mask, float scale, void* dQ, void* dK, void* dV,
