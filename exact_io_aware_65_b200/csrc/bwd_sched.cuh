@@ -40,6 +40,17 @@ struct Params {
   uint32_t* status;
 };
 
+// Heads per scheduling group.  The group's Q and dO tiles (bf16) and fp32
+// dQ accumulator rows are the backward's working set in L2, kept to about
+// 64 MiB; at least 8 heads, or all of them (short sequences: one group,
+// whose longest-first order then evens out the CTAs' work).
+__host__ __device__ inline int sched_group(int BH, int N, int d) {
+  const long long per_head = 8LL * (N > 0 ? N : 1) * d;  // Q, dO bf16 and the fp32 dQ rows
+  const long long fit = (64LL << 20) / per_head;
+  const long long g = fit > 8 ? fit : 8;
+  return (int)(g < BH ? g : BH);
+}
+
 struct Item {
   int bh, j;
   int Lq, Lk, off, nqb;  // this sequence's query rows and keys, causal offset, query tiles

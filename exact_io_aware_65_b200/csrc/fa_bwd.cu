@@ -976,7 +976,7 @@ static fa_status launch_bwd_d(const Problem& pr, const CUtensorMap& mQ, const CU
     p.sched = sched;
     p.turn = turn;
     p.deterministic = pr.deterministic;
-    p.group = pr.BH < 8 ? pr.BH : 8;
+    p.group = bwd::sched_group(pr.BH, pr.N, pr.d);
     p.dK = static_cast<__nv_bfloat16*>(dK);
     p.dV = static_cast<__nv_bfloat16*>(dV);
     p.timeout_ns = wait_timeout_ns();

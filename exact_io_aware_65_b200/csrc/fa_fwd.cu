@@ -720,7 +720,7 @@ fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void
   p.tiles_per_item = dual ? 1 : 2;
   p.n_pairs = (pr.nq + p.tiles_per_item - 1) / p.tiles_per_item;
   p.n_items = p.n_pairs * pr.BH;
-  p.group = pr.BH < 8 ? pr.BH : 8;
+  p.group = fwd::sched_group(pr.BH, pr.Nk, pr.d);
   p.mask_kind = pr.mask_kind;
   p.block_mask = pr.block_mask;
   p.scale_log2 = pr.scale_log2;

@@ -38,6 +38,18 @@ struct Params {
   uint32_t slot;  // scheduler counter slot of this launch
 };
 
+// Heads per scheduling group.  The group's K and V tiles are the forward's
+// working set in L2, kept to about 32 MiB; above that, more heads per group
+// spread the longest-first order over more items, which evens out the CTAs'
+// work under a causal mask (short sequences: all heads in one group).  At
+// least 8 heads, or all of them.
+__host__ __device__ inline int sched_group(int BH, int Nk, int d) {
+  const long long per_head = 4LL * (Nk > 0 ? Nk : 1) * d;  // K and V, bf16
+  const long long fit = (32LL << 20) / per_head;
+  const long long g = fit > 8 ? fit : 8;
+  return (int)(g < BH ? g : BH);
+}
+
 struct Item {
   int bh, q0, q1;
   bool has1;

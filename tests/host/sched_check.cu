@@ -64,7 +64,7 @@ void fail(const char* what, const Problem& pr, int a, int b, int c) {
 }
 
 template <bool VARLEN>
-void check_fwd(const Problem& pr, int tiles_per_item) {
+void check_fwd(const Problem& pr, int tiles_per_item, int group) {
   using namespace fa::fwd;
   Params p = {};
   p.tiles_per_item = tiles_per_item;
@@ -74,7 +74,7 @@ void check_fwd(const Problem& pr, int tiles_per_item) {
   p.seqlens_k = VARLEN ? pr.lk.data() : nullptr;
   p.n_pairs = (p.nq + tiles_per_item - 1) / tiles_per_item;
   p.n_items = p.n_pairs * BH;
-  p.group = BH < 8 ? BH : 8;
+  p.group = group;
   p.mask_kind = pr.kind;
   p.block_mask = pr.kind == FA_MASK_BLOCK ? pr.mask.data() : nullptr;
   p.status = &g_status;
@@ -109,7 +109,7 @@ void check_fwd(const Problem& pr, int tiles_per_item) {
 }
 
 template <bool VARLEN>
-void check_bwd(const Problem& pr) {
+void check_bwd(const Problem& pr, int group) {
   using namespace fa::bwd;
   Params p = {};
   const int BH = pr.B * pr.H;
@@ -120,7 +120,7 @@ void check_bwd(const Problem& pr) {
   p.n_items = BH * p.nk;
   p.mask_kind = pr.kind;
   p.block_mask = pr.kind == FA_MASK_BLOCK ? pr.mask.data() : nullptr;
-  p.group = BH < 8 ? BH : 8;
+  p.group = group;
   p.status = &g_status;
   std::vector<int> owner((size_t)BH * p.nk, 0);
   // visits[bh][i] = key tiles that visit query tile i, in ascending order
@@ -186,13 +186,25 @@ int main() {
                   pr.lq.push_back(u == 0 ? 0 : u == 1 ? pr.Nq : (int)(rnd() % (pr.Nq + 1)));
                   pr.lk.push_back(u == 0 ? pr.Nk : u == 1 ? pr.Nk : (int)(rnd() % (pr.Nk + 1)));
                 }
-                check_fwd<true>(pr, 2);
-                check_fwd<true>(pr, 1);
-                check_bwd<true>(pr);
-              } else {
-                check_fwd<false>(pr, 2);
-                check_fwd<false>(pr, 1);
-                check_bwd<false>(pr);
+              }
+              // the launches' own group sizes for this shape lie in [1, BH];
+              // the schedules are walked for those and for every other size
+              // from one head to all of them
+              const int BH = B * H;
+              const int own[] = {fa::fwd::sched_group(BH, pr.Nk, 64), fa::fwd::sched_group(BH, pr.Nk, 128),
+                                 fa::bwd::sched_group(BH, pr.Nq, 64), fa::bwd::sched_group(BH, pr.Nq, 128)};
+              for (int g : own)
+                if (g < 1 || g > BH) { fail("group size out of range", pr, g, BH, 0); return 1; }
+              for (int g = 1; g <= BH; ++g) {
+                if (var) {
+                  check_fwd<true>(pr, 2, g);
+                  check_fwd<true>(pr, 1, g);
+                  check_bwd<true>(pr, g);
+                } else {
+                  check_fwd<false>(pr, 2, g);
+                  check_fwd<false>(pr, 1, g);
+                  check_bwd<false>(pr, g);
+                }
               }
               ++cases;
               if (g_fail) return 1;

@@ -2,8 +2,9 @@
 
 tests/host/sched_check.cu includes the very functions the kernels use to
 pick their tiles (fwd_sched.cuh, bwd_sched.cuh, host-callable), walks every
-work item of 2916 problems, and compares the tiles visited with the
-visibility rule written row by row.  The problems cover ragged and unequal
+work item of 2916 problems, at every head-group size from one head to all
+of them, and compares the tiles visited with the visibility rule written row
+by row.  The group sizes the launches choose must lie in that range.  The problems cover ragged and unequal
 query and key counts, all masks, random block masks with empty rows and
 columns, and per-sequence lengths.  It also checks the order the
 deterministic backward adds dQ in.  Planted mistakes in copies of the
