@@ -7,7 +7,7 @@
 // values past it, and keep a running row maximum and row sum so that the
 // softmax is completed incrementally; the N x N scores live only on chip.
 //
-// B200 mapping (one persistent CTA per SM, 384 threads):
+// B200 mapping (one persistent CTA per SM, 384 threads), d = 128:
 //   warp 0        TMA producer: two 128-row Q tiles per work item, then a ring
 //                 of K and V tiles (128 keys x d, 128-byte swizzle).
 //   warps 1(, 2)  MMA issuer(s), one thread each (Cfg::ISSUERS): S_t = Q_t K_j^T
@@ -18,10 +18,9 @@
 //                 tensor memory, keeps the row max m and row sum l in
 //                 registers, writes P (bf16) into tensor memory, and does
 //                 the final O / l and LSE epilogue.
-// At d = 64 under a block mask the CTA runs two independent pipelines
-// (Cfg::DUAL): warps 0 and 3 produce, 1 and 2 issue, 4..7 and 8..11 do the
-// softmax, each pipeline with its own Q tile, K/V ring and work items of one
-// query tile.
+// At d = 64 the CTA runs two independent pipelines (Cfg::DUAL): warps 0 and
+// 3 produce, 1 and 2 issue, 4..7 and 8..11 do the softmax, each pipeline with
+// its own Q tile, K/V ring and work items of one query tile.
 // Tensor memory (512 columns):
 //   d = 128: S/P of tile t at [128 t, 128 t + 128) (P, bf16, over the scores),
 //            O of tile t at [256 + 128 t, 384 + 128 t).  A tile's next QK^T
@@ -72,18 +71,17 @@ struct Cfg {
   static constexpr int TILE_BYTES = BN * D * 2;  // one Q, K or V tile
   static constexpr int CHUNKS = D / 64;          // 64-column (128-byte) chunks per row
   static constexpr int CHUNK_BYTES = BN * 128;   // one chunk of a tile
-  // PIPES = 2 (d = 64 under a block mask): two independent pipelines per
-  // CTA.  Each has its own producer warp (0, 3), MMA issuer (1, 2), softmax
-  // warpgroup (4..7, 8..11), Q tile, K/V ring and stream of work items, one
-  // query tile each; they share only the CTA's shared and tensor memory, so
-  // one pipeline's softmax, item change or load wait overlaps the other's
-  // work, and neither loads key tiles only the other needs.  PIPES = 1: one
-  // pipeline, work items of two query tiles sharing one K/V stream (better
-  // where the two tiles need the same key tiles: no mask, causal).
-  static_assert(PIPES == 1 || (PIPES == 2 && D == 64), "two pipelines need the d = 64 column plan");
+  // PIPES = 2 (d = 64): two independent pipelines per CTA.  Each has its own
+  // producer warp (0, 3), MMA issuer (1, 2), softmax warpgroup (4..7,
+  // 8..11), Q tile, K/V ring and stream of work items, one query tile each;
+  // they share only the CTA's shared and tensor memory, so one pipeline's
+  // softmax, item change or load wait overlaps the other's work, and neither
+  // loads key tiles only the other needs.  PIPES = 1 (d = 128): one
+  // pipeline, work items of two query tiles sharing one K/V stream.
+  static_assert(PIPES == (D == 64 ? 2 : 1), "d = 64 runs two pipelines, d = 128 one");
   static constexpr bool DUAL = PIPES == 2;
   static constexpr int NPIPE = PIPES;
-  static constexpr int NSLOT = DUAL ? 4 : (D == 64 ? 8 : 4);  // K/V ring slots per pipeline
+  static constexpr int NSLOT = 4;  // K/V ring slots per pipeline
   // Each softmax warp stages 64 columns of its 32 rows of O (bf16, 4 KB) at
   // a time here, in the 128-byte swizzle, and writes them out with one
   // tensor store.
@@ -91,7 +89,7 @@ struct Cfg {
   static constexpr int SMEM_BYTES = 2 * TILE_BYTES + NPIPE * NSLOT * TILE_BYTES + OSTAGE_BYTES + 1024;
   // MMA issuer threads.  Issuing blocks while the tensor core's queue is
   // full, so with one issuer a tile's PV can wait behind the other tile's
-  // products.  d = 64: one issuer per query tile (short products, so the
+  // products.  d = 64: one issuer per pipeline (short products, so the
   // decoupling wins).  d = 128: one issuer for both tiles, which keeps each
   // tile's PV and next QK^T back to back on the tensor core (interleaving
   // the two tiles' products delays both tiles' next scores).
@@ -715,8 +713,8 @@ fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void
   p.H = pr.H;
   p.seqlens_q = pr.seqlens_q;
   p.seqlens_k = pr.seqlens_k;
-  // d = 64 under a block mask: two pipelines of one-tile items
-  const bool dual = pr.d == 64 && pr.mask_kind == FA_MASK_BLOCK;
+  // d = 64: two pipelines of one-tile items; d = 128: pairs
+  const bool dual = pr.d == 64;
   p.tiles_per_item = dual ? 1 : 2;
   p.n_pairs = (pr.nq + p.tiles_per_item - 1) / p.tiles_per_item;
   p.n_items = p.n_pairs * pr.BH;
@@ -740,12 +738,9 @@ fa_status launch_fwd(const Problem& pr, const void* Q, const void* K, const void
   };
   const bool varlen = pr.seqlens_q || pr.seqlens_k;
   bool ok;
-  if (pr.d == 64 && dual)
+  if (dual)
     ok = varlen ? run(fwd::fwd_kernel<64, true, 2>, fwd::Cfg<64, 2>::SMEM_BYTES)
                 : run(fwd::fwd_kernel<64, false, 2>, fwd::Cfg<64, 2>::SMEM_BYTES);
-  else if (pr.d == 64)
-    ok = varlen ? run(fwd::fwd_kernel<64, true, 1>, fwd::Cfg<64, 1>::SMEM_BYTES)
-                : run(fwd::fwd_kernel<64, false, 1>, fwd::Cfg<64, 1>::SMEM_BYTES);
   else
     ok = varlen ? run(fwd::fwd_kernel<128, true, 1>, fwd::Cfg<128, 1>::SMEM_BYTES)
                 : run(fwd::fwd_kernel<128, false, 1>, fwd::Cfg<128, 1>::SMEM_BYTES);
