@@ -165,6 +165,20 @@ uint32_t rnd() {  // xorshift64
 }  // namespace
 
 int main() {
+  // The group sizes the launches choose for the benchmark shapes: 8 heads
+  // where a head's tiles are large (long causal, block-sparse), every head
+  // where they are small (BERT- and GPT-2-shaped).
+  struct GroupCase { int BH, N, d, fwd, bwd; };
+  const GroupCase gc[] = {{32, 8192, 128, 8, 8}, {8, 16384, 64, 8, 8}, {256, 512, 64, 256, 256},
+                          {96, 1024, 64, 96, 96}, {3, 100, 64, 3, 3}, {1000, 65536, 128, 8, 8}};
+  for (const GroupCase& c : gc) {
+    const int f = fa::fwd::sched_group(c.BH, c.N, c.d), b = fa::bwd::sched_group(c.BH, c.N, c.d);
+    if (f != c.fwd || b != c.bwd) {
+      printf("MISMATCH group size for BH=%d N=%d d=%d: fwd %d (want %d), bwd %d (want %d)\n", c.BH, c.N, c.d, f,
+             c.fwd, b, c.bwd);
+      return 1;
+    }
+  }
   const int sizes[] = {1, 100, 127, 128, 129, 256, 300, 640, 1000};
   const int nsz = sizeof(sizes) / sizeof(sizes[0]);
   long cases = 0;
