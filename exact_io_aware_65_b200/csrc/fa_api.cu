@@ -93,8 +93,11 @@ using namespace fa;
 
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// The kernels count work items (heads x 128-row tiles) and tile rows in
+// 32-bit ints: B*H*N up to 2^37 keeps both below 2^31 (and is far beyond
+// what fits in device memory at d = 64).
 static bool sizes_supported(long long bh, int N) {
-  return bh <= (1ll << 30) && N <= (1 << 30) && bh * (long long)N <= (1ll << 40);
+  return bh <= (1ll << 30) && N <= (1 << 30) && bh * (long long)N <= (1ll << 37);
 }
 
 static fa_status check_common(const void* Q, const void* K, const void* V, int B, int H, int N, int Nk, int d,

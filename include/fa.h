@@ -60,7 +60,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, bad scale, bad mask kind */
-  FA_ERR_UNSUPPORTED = 2, /* valid request outside this build: d not 64/128, sizes beyond int range */
+  FA_ERR_UNSUPPORTED = 2, /* valid request outside this build: d not 64/128, B*H*N or B*H*Nk above 2^37 */
   FA_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed */
   FA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than fa_bwd_workspace_size() */
   FA_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out (see fa_device_status) */

@@ -59,6 +59,8 @@ def test_workspace_size_is_linear_in_sequence_length():
     assert s1 > 0 and abs(s2 / s1 - 2.0) < 1e-3
     assert fa.bwd_workspace_size(1, 1, 100, 96) == 0
     assert fa.bwd_workspace_size(0, 1, 100, 64) == 0
+    assert fa.bwd_workspace_size(1 << 20, 1 << 10, 1 << 10, 64) == 0   # B*H*N > 2^37
+    assert fa.bwd_workspace_size(1 << 10, 1 << 10, 1 << 17, 64) > 0     # B*H*N = 2^37
 
 
 FAKE = 1 << 20  # a 16-byte aligned non-null address; never dereferenced
@@ -75,6 +77,7 @@ FAKE = 1 << 20  # a 16-byte aligned non-null address; never dereferenced
     (dict(mask=2, bm=0), 1),            # block mask missing
     (dict(Q=FAKE + 8), 1),              # misaligned
     (dict(d=96), 2),                    # head size not supported
+    (dict(B=1 << 20, H=1 << 10, N=1 << 10), 2),   # B*H*N beyond 32-bit work-item counts
 ])
 def test_fwd_rejects_bad_arguments_on_host(args, code):
     a = dict(Q=FAKE, K=FAKE, V=FAKE, B=1, H=1, N=128, d=64, mask=0, bm=0, scale=0.125, O=FAKE, L=FAKE)
